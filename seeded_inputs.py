@@ -1,0 +1,109 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module holds the workload shapes and the random draws only -- none of
+the attention arithmetic -- so that the CUDA path and the fp64 oracle are fed
+bit-identical fp16/bf16 values without sharing any code.
+
+Recipe: a CPU ``torch.Generator`` seeded with the workload's seed draws
+``torch.randn`` in fp32, in the order Q, K, V, then dO, each in the
+``[batch, seq, heads, head_dim]`` layout of ``flash_attn_func``
+("optimizing-attention-flash", Workflow 2, Step 2); the fp32 draws are then
+rounded once to the workload dtype.  Values are i.i.d. N(0, 1), as in the
+pages' own benchmark and accuracy snippets (``torch.randn``, Workflow 1
+Steps 3-4).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    seqlen_q: int
+    seqlen_k: int
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    dtype: torch.dtype
+    causal: bool
+    window: tuple = (-1, -1)
+    seed: int = 0
+    backward: bool = False
+    note: str = field(default="", compare=False)
+
+    @property
+    def softmax_scale(self) -> float:
+        # the pages' default: 1 / sqrt(head_dim)
+        return float(self.head_dim) ** -0.5
+
+    def describe(self) -> dict:
+        return {
+            "workload": self.name, "batch": self.batch, "seqlen_q": self.seqlen_q,
+            "seqlen_k": self.seqlen_k, "q_heads": self.q_heads, "kv_heads": self.kv_heads,
+            "head_dim": self.head_dim, "dtype": str(self.dtype).replace("torch.", ""),
+            "causal": self.causal, "window_size": list(self.window), "seed": self.seed,
+            "backward": self.backward,
+        }
+
+
+F16, BF16 = torch.float16, torch.bfloat16
+
+# The five workloads of the pages' benchmark plan; shapes of 2 and 3 restate the
+# pages' own benchmark snippets ("optimizing-attention-flash", Workflow 1 Step 3
+# at 2x8x2048x64 and Workflow 2 Step 4 at 4x32x4096x64).
+WORKLOADS = {
+    "tiny_128_d64_fp16": Workload("tiny_128_d64_fp16", 1, 128, 128, 2, 2, 64, F16, False, seed=0),
+    "fwd_2x2048_h8_d64_fp16": Workload("fwd_2x2048_h8_d64_fp16", 2, 2048, 2048, 8, 8, 64, F16,
+                                       False, seed=1),
+    "fwd_2x2048_h8_d64_fp16_causal": Workload("fwd_2x2048_h8_d64_fp16_causal", 2, 2048, 2048, 8,
+                                              8, 64, F16, True, seed=1),
+    "fwd_4x4096_h32_d64_fp16_causal": Workload("fwd_4x4096_h32_d64_fp16_causal", 4, 4096, 4096,
+                                               32, 32, 64, F16, True, seed=2),
+    "fwd_2x4096_h32kv8_d128_bf16_causal_win256": Workload(
+        "fwd_2x4096_h32kv8_d128_bf16_causal_win256", 2, 4096, 4096, 32, 8, 128, BF16, True,
+        window=(256, 0), seed=3),
+    "fwdbwd_1x16384_h16_d128_bf16_causal": Workload("fwdbwd_1x16384_h16_d128_bf16_causal", 1,
+                                                    16384, 16384, 16, 16, 128, BF16, True,
+                                                    seed=4, backward=True),
+}
+
+
+def make_qkv(batch, seqlen_q, seqlen_k, q_heads, kv_heads, head_dim, dtype, seed,
+             with_dout=False):
+    """Q, K, V (and dO) as CPU tensors of ``dtype``, drawn in the order Q, K, V, dO."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((batch, seqlen_q, q_heads, head_dim), generator=g, dtype=torch.float32)
+    k = torch.randn((batch, seqlen_k, kv_heads, head_dim), generator=g, dtype=torch.float32)
+    v = torch.randn((batch, seqlen_k, kv_heads, head_dim), generator=g, dtype=torch.float32)
+    out = [q.to(dtype), k.to(dtype), v.to(dtype)]
+    if with_dout:
+        do = torch.randn((batch, seqlen_q, q_heads, head_dim), generator=g, dtype=torch.float32)
+        out.append(do.to(dtype))
+    return tuple(out)
+
+
+def make_workload_inputs(w: Workload, with_dout=None):
+    if with_dout is None:
+        with_dout = w.backward
+    return make_qkv(w.batch, w.seqlen_q, w.seqlen_k, w.q_heads, w.kv_heads, w.head_dim, w.dtype,
+                    w.seed, with_dout=with_dout)
+
+
+def sample_rows(batch, q_heads, seqlen_q, n, seed):
+    """n distinct (b, h, i) triples, always including the first and last row of
+    the sequence so the ragged tail and the causal corner are covered."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7919)
+    b = torch.randint(0, batch, (n,), generator=g)
+    h = torch.randint(0, q_heads, (n,), generator=g)
+    i = torch.randint(0, seqlen_q, (n,), generator=g)
+    i[0] = 0
+    if n > 1:
+        i[1] = seqlen_q - 1
+    rows = torch.stack([b, h, i], dim=1)
+    return torch.unique(rows, dim=0).numpy()
