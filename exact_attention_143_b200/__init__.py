@@ -1,0 +1,191 @@
+"""Python binding of libfa143.so, the B200 (sm_100a) exact-attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/fa143.h.  PyTorch provides the
+device memory and the current stream.  There is no fallback: if the shared
+library is missing or a tensor is not on a CUDA device the call raises.
+
+    o, lse = fa_fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1))
+    dq, dk, dv = fa_bwd(do, q, k, v, o, lse, softmax_scale=None, causal=False,
+                        window_size=(-1, -1))
+
+Tensors use the [batch, seqlen, heads, head_dim] layout and fp16/bf16 of
+flash_attn_func ("optimizing-attention-flash", Workflow 2 Steps 2-3);
+softmax_scale=None means 1/sqrt(head_dim); k and v may have fewer heads than
+q (MQA/GQA); window_size=(left, right) with -1 for unbounded.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa143.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_ALIGNMENT = 3
+FA_ERR_WORKSPACE = 4
+FA_ERR_CUDA = 5
+FA_ERR_DEVICE_TIMEOUT = 6
+
+# names exported by libfa143.so (the declarations of include/fa143.h)
+EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
+            "fa_get_device_error", "fa_set_wait_limit_ns")
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libfa143.so and declare its C signatures (no GPU needed)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libfa143.so is not built (%s); run exact_attention_143_b200.build"
+                           ".build() or __graft_entry__.build()" % path)
+    lib = ctypes.CDLL(path)
+    vp, i, f, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_int64)
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i64p, i64p, i64p, i64p, i, f, i,
+                           i, i, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_bwd.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [i] * 6 + [i64p] * 8 +
+                           [i, f, i, i, i, vp])
+    lib.fa_bwd.restype = i
+    lib.fa_get_device_error.argtypes = [vp]
+    lib.fa_get_device_error.restype = i
+    lib.fa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.fa_set_wait_limit_ns.restype = ctypes.c_uint64
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().fa_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return 0
+    if t.dtype == torch.bfloat16:
+        return 1
+    raise TypeError("fp16 or bf16 tensors only (got %s)" % t.dtype)
+
+
+def _strides(t: torch.Tensor):
+    if t.dim() != 4:
+        raise ValueError("expected a [batch, seqlen, heads, head_dim] tensor, got shape %s"
+                         % (tuple(t.shape),))
+    if t.stride(3) != 1 and t.shape[3] > 1:
+        raise ValueError("head_dim must be contiguous (stride 1)")
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _check_cuda(*ts):
+    dev = ts[0].device
+    for t in ts:
+        if not t.is_cuda:
+            raise RuntimeError("tensors must be on a CUDA device (no CPU path exists)")
+        if t.device != dev:
+            raise RuntimeError("all tensors must be on the same device")
+    return dev
+
+
+def _scale(softmax_scale, d):
+    return 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def fa_fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), out=None, lse=None):
+    """Exact attention forward; returns (o [B,Nq,Hq,d], lse [B,Hq,Nq] fp32)."""
+    lib = load_library()
+    dev = _check_cuda(q, k, v)
+    code = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty((B, Nq, Hq, d), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+    _check_cuda(q, out, lse)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Nq] tensor")
+    wl, wr = window_size
+    with torch.cuda.device(dev):
+        rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                        B, Nq, Nk, Hq, Hkv, d, _strides(q), _strides(k), _strides(v),
+                        _strides(out), code, _scale(softmax_scale, d), int(bool(causal)),
+                        int(wl), int(wr), _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_fwd")
+    return out, lse
+
+
+def bwd_workspace_size(B, Nq, Hq, d) -> int:
+    return int(load_library().fa_bwd_workspace_size(B, Nq, Hq, d))
+
+
+def fa_bwd(dout, q, k, v, o, lse, softmax_scale=None, causal=False, window_size=(-1, -1),
+           dq=None, dk=None, dv=None, workspace=None):
+    """Exact attention backward from the forward's O and LSE; returns (dq, dk, dv)."""
+    lib = load_library()
+    dev = _check_cuda(dout, q, k, v, o, lse)
+    code = _dtype_code(q)
+    for t in (k, v, o, dout):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, o, dout must share one dtype")
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be the contiguous fp32 [B, Hq, Nq] tensor from fa_fwd")
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    ws_bytes = bwd_workspace_size(B, Nq, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    _check_cuda(q, dq, dk, dv, workspace)
+    wl, wr = window_size
+    with torch.cuda.device(dev):
+        rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                        lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                        B, Nq, Nk, Hq, Hkv, d, _strides(q), _strides(k), _strides(v),
+                        _strides(o), _strides(dout), _strides(dq), _strides(dk), _strides(dv),
+                        code, _scale(softmax_scale, d), int(bool(causal)), int(wl), int(wr),
+                        _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def get_device_error(device=None) -> int:
+    """Synchronise the current stream and return/clear the device error word."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(lib.fa_get_device_error(_stream(dev)))
+
+
+def set_wait_limit_ns(limit_ns: int) -> int:
+    return int(load_library().fa_set_wait_limit_ns(int(limit_ns)))

@@ -1,0 +1,143 @@
+/*
+ * fa143.h -- C ABI of the B200 (sm_100a) exact-attention library libfa143.so.
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(Q K^T * softmax_scale + mask) V
+ *
+ * ("optimizing-attention-flash", Workflow 1 Step 2: the standard-attention
+ * form softmax(q k^T / sqrt(d_k)) v that the fused kernel replaces) tile by
+ * tile, so the N x N score matrix never reaches HBM ("Что такое
+ * FlashAttention…", section "Основной механизм простыми словами": blocks of
+ * Q, K, V are brought from HBM into on-chip memory, attention is computed per
+ * block and the output is updated incrementally; the result is exact, without
+ * approximation).  The backward pass rebuilds the probabilities from the
+ * per-row log-sum-exp saved by the forward ("tiling and recomputation",
+ * "optimizing-attention-flash", Quick start).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors use the [batch, seqlen, heads, head_dim] layout of
+ *    flash_attn_func ("optimizing-attention-flash", Workflow 2 Step 2).
+ *    Each tensor is described by a device pointer plus three strides, in
+ *    ELEMENTS, for (batch, seq, head); head_dim is contiguous (stride 1).
+ *    Pointers must be 16-byte aligned and the three strides must be
+ *    multiples of 8 elements (16 bytes), as the tensor-memory-accelerator
+ *    copies require; otherwise FA_ERR_ALIGNMENT.
+ *  - dtype is FA_F16 or FA_BF16 for every tensor of one call; fp32 inputs
+ *    are not supported (the pages' troubleshooting section: fp16/bf16 only).
+ *  - head_dim d is 64 or 128.
+ *  - Hq query heads, Hkv key/value heads, Hq % Hkv == 0: query head h reads
+ *    kv head h / (Hq / Hkv) (MQA/GQA, Workflow 2 Step 3).
+ *  - causal != 0 hides key j from query i when j > i + (Nk - Nq) (masks are
+ *    aligned to the bottom-right corner when Nq != Nk).  window_left /
+ *    window_right >= 0 keep only keys with
+ *        i + (Nk - Nq) - window_left <= j <= i + (Nk - Nq) + window_right
+ *    (bounds inclusive); -1 means unbounded on that side (Workflow 2
+ *    Step 3's window_size=(left, right), (-1, -1) = no window).  causal and
+ *    a window combine as the intersection.
+ *  - A query row that sees no key gets O = 0 and LSE = -inf, and zero dQ.
+ *  - softmax_scale is passed explicitly and must be finite (the Python
+ *    binding maps "None" to 1/sqrt(head_dim), Workflow 2 Step 2).
+ *  - LSE is float32, contiguous [batch, Hq, Nq], natural logarithm of
+ *    sum_j exp(softmax_scale * q_i . k_j) over the visible keys.
+ *  - Everything is asynchronous on `stream` (a cudaStream_t passed as a void
+ *    pointer; NULL = legacy default stream).  Errors are returned as status
+ *    codes, never thrown; argument errors are detected on the host before any
+ *    launch.  The caller owns every buffer; outputs must not alias inputs.
+ *  - Device-side waits are bounded: a kernel whose pipeline stalls past the
+ *    limit records FA_ERR_DEVICE_TIMEOUT in a device error word and returns;
+ *    read it with fa_get_device_error().
+ */
+#ifndef FA143_H
+#define FA143_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
+
+enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad window, Hq % Hkv != 0, aliasing */
+    FA_ERR_UNSUPPORTED = 2,    /* dtype or head_dim outside what the kernels implement */
+    FA_ERR_ALIGNMENT = 3,      /* pointer or stride violates the 16-byte rules above */
+    FA_ERR_WORKSPACE = 4,      /* backward workspace missing or too small */
+    FA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or a launch failed */
+    FA_ERR_DEVICE_TIMEOUT = 6  /* a bounded device-side wait ran out (see fa_get_device_error) */
+};
+
+/* Human-readable text of a status code (static storage, never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * Forward pass: O and the per-row LSE.
+ *   q      [B, Nq, Hq, d]   read-only     strides q_stride = {batch, seq, head}
+ *   k, v   [B, Nk, Hkv, d]  read-only     strides k_stride, v_stride
+ *   o      [B, Nq, Hq, d]   written       strides o_stride
+ *   lse    [B, Hq, Nq] fp32 written       contiguous
+ * One kernel launch on `stream`.  Returns FA_OK or an error status.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int Nq, int Nk, int Hq, int Hkv, int d,
+           const int64_t q_stride[3], const int64_t k_stride[3],
+           const int64_t v_stride[3], const int64_t o_stride[3],
+           int dtype, float softmax_scale, int causal, int window_left,
+           int window_right, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
+ * accumulator [B, Nq, Hq, d] and the fp32 row terms D and LSE*log2(e)
+ * [B, Hq, Nq].  The caller allocates it (256-byte aligned); its contents
+ * on entry do not matter.
+ */
+size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d);
+
+/*
+ * Backward pass: dQ, dK, dV of L = sum(dout * O), recomputing the
+ * probabilities from the forward's LSE (the textbook gradient of the
+ * definition above: dV = P^T dO, dP = dO V^T, D = rowsum(dO * O),
+ * dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q; the query heads of
+ * one GQA group are summed into their shared kv head).
+ *   q, o, dout [B, Nq, Hq, d]  read-only   (o and lse from fa_fwd with the
+ *   k, v       [B, Nk, Hkv, d] read-only    same arguments)
+ *   lse        [B, Hq, Nq] fp32 read-only
+ *   dq         [B, Nq, Hq, d]  written
+ *   dk, dv     [B, Nk, Hkv, d] written
+ *   workspace  >= fa_bwd_workspace_size(B, Nq, Hq, d) bytes, device memory
+ * Launches a short sequence of kernels on `stream`.  dQ is accumulated with
+ * fp32 atomics, so its last bits may differ from run to run.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, void* workspace,
+           size_t workspace_bytes,
+           int B, int Nq, int Nk, int Hq, int Hkv, int d,
+           const int64_t q_stride[3], const int64_t k_stride[3],
+           const int64_t v_stride[3], const int64_t o_stride[3],
+           const int64_t do_stride[3], const int64_t dq_stride[3],
+           const int64_t dk_stride[3], const int64_t dv_stride[3],
+           int dtype, float softmax_scale, int causal, int window_left,
+           int window_right, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of
+ * the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel gave up
+ * on a bounded wait since the last call (FA_ERR_CUDA if the query failed).
+ */
+int fa_get_device_error(void* stream);
+
+/*
+ * Sets the per-wait limit of device-side waits, in nanoseconds (default
+ * 2e9).  Returns the previous value.  For tests of the timeout path only.
+ */
+uint64_t fa_set_wait_limit_ns(uint64_t limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA143_H */
