@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention library on B200.
+
+One step = one forward (fa_fwd) plus one backward (fa_bwd) over the
+long-context workload: batch 1, 16 heads, 16384 tokens, head_dim 128, bf16,
+causal; Q, K, V, dO i.i.d. N(0, 1) from a seeded CPU generator (synthetic).
+That step runs every stage of the hot path: tile planning, the TMA/tcgen05
+forward with online softmax and the LSE epilogue, the backward preprocess,
+the recomputing backward main kernel and the dQ conversion.
+
+Metric: attention TFLOPS of the fwd+bwd step, counting 4*B*Hq*d per visible
+(query, key) pair forward and 2.5x that backward (masked work not counted),
+whole job over all ranks.  L2 is flushed (256 MB write) before every timed
+step; each step is timed with its own CUDA events on the launching stream.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) every rank runs an independent replica (weak scaling,
+no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from seeded_inputs import WORKLOADS, Workload, make_qkv, make_workload_inputs  # noqa: E402
+
+METRIC = "attention TFLOPS (fwd, fwd+bwd) on 1 B200 and % of dense FP16/BF16 tensor peak"
+MAIN_WORKLOAD = "fwdbwd_1x16384_h16_d128_bf16_causal"
+FWD_TABLE = ["fwd_2x2048_h8_d64_fp16", "fwd_2x2048_h8_d64_fp16_causal",
+             "fwd_4x4096_h32_d64_fp16_causal", "fwd_2x4096_h32kv8_d128_bf16_causal_win256"]
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- counting
+def visible_pairs(Nq, Nk, causal, window):
+    """Number of (query, key) pairs the mask keeps, per (batch, head)."""
+    i = np.arange(Nq, dtype=np.int64)
+    ip = i + (Nk - Nq)
+    wl, wr = window
+    right = 0 if causal else wr
+    lo = np.maximum(0, ip - wl) if wl >= 0 else np.zeros_like(ip)
+    hi = np.minimum(Nk - 1, ip + right) if right >= 0 else np.full_like(ip, Nk - 1)
+    return int(np.maximum(hi - lo + 1, 0).sum())
+
+
+def fwd_flops(w: Workload):
+    """Forward FLOPs: 4 * batch * q_heads * head_dim per visible pair."""
+    return 4.0 * w.batch * w.q_heads * w.head_dim * \
+        visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("fa_bwd.cuh", "fa_fwd.cuh", "fa_ptx.cuh", "fa143_api.cu"):
+        with open(os.path.join(ROOT, "exact_attention_143_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    if it was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tr = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = tr.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.rows = []
+        self.proc = None
+
+    def _gpu_id(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            return str(self.dev)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self._gpu_id(), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for k, nm in enumerate(names):
+                if r[5 + k].lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample_rate(w: Workload, budget_s: float):
+    """Time the fp64 oracle (fwd + bwd) on a prefix of one head of workload w,
+    sized to take about budget_s; returns (TFLOPS, sample description, cores)."""
+    import oracle
+
+    def run(T):
+        q, k, v, do = make_qkv(1, T, T, 1, 1, w.head_dim, w.dtype, w.seed, with_dout=True)
+        f = lambda t: t.float().double().numpy()  # noqa: E731
+        t0 = time.perf_counter()
+        oracle.attention_fwd(f(q), f(k), f(v), w.softmax_scale, w.causal, w.window)
+        oracle.attention_bwd(f(q), f(k), f(v), f(do), w.softmax_scale, w.causal, w.window)
+        dt = time.perf_counter() - t0
+        flops = 3.5 * 4.0 * w.head_dim * visible_pairs(T, T, w.causal, w.window)
+        return dt, flops
+
+    T = min(512, w.seqlen_q)
+    dt, flops = run(T)
+    # the oracle's cost grows with the pair count, about T^2
+    T = int(min(w.seqlen_q, max(T, T * math.sqrt(max(budget_s, 0.1) / max(dt, 1e-3)))))
+    T = max(128, T // 128 * 128)
+    dt, flops = run(T)
+    sample = ("fp64 oracle fwd+bwd on the first %d tokens of one (batch, head) of %s "
+              "(%.3g algorithmic GFLOP in %.2f s)" % (T, w.name, flops / 1e9, dt))
+    import oracle as _o
+    return flops / dt / 1e12, sample, _o.default_threads(), T, dt
+
+
+# ---------------------------------------------------------------- our arm
+def time_steps(step, K, W, flush, stream, per_step_events=None):
+    """Run W warm-up steps, then K steps each bracketed by its own events, with
+    an L2 flush before every step (outside the events).  Returns ms per step list."""
+    for _ in range(W):
+        flush()
+        step(None)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for i in range(K):
+        flush()
+        evs[i][0].record(stream)
+        step(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def run_ours(args):
+    import exact_attention_143_b200 as fa
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOADS[args.workload]
+    peaks, peak_src = load_peaks()
+
+    # inputs (each rank an independent replica: seed + rank), resident in HBM
+    wr = Workload(**{**w.__dict__, "seed": w.seed + rank})
+    q, k, v, do = make_workload_inputs(wr, with_dout=True)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty(w.batch, w.q_heads, w.seqlen_q, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(fa.bwd_workspace_size(w.batch, w.seqlen_q, w.q_heads, w.head_dim),
+                     dtype=torch.uint8, device=dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = lambda: flush_buf.zero_()  # noqa: E731
+    kw = dict(softmax_scale=w.softmax_scale, causal=w.causal, window_size=w.window)
+
+    K, W = args.steps, args.warmup
+    main_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    for a, b in main_ev:  # materialise the events before handing them to the library
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+
+    def step(i):
+        if i is not None:
+            fa.set_bwd_main_events(*main_ev[i])
+        else:
+            fa.set_bwd_main_events(None, None)
+        fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw)
+        fa.fa_bwd(dod, qd, kd, vd, o, lse, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+
+    clocks = ClockSampler(local)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall0 = time.perf_counter()
+    ms = time_steps(step, K, W, flush, stream)
+    t_wall = time.perf_counter() - t_wall0
+    clk = clocks.stop()
+    fa.set_bwd_main_events(None, None)
+    dist_barrier(world)
+    assert fa.get_device_error(dev) == fa.FA_OK
+    main_ms = [a.elapsed_time(b) for a, b in main_ev]
+
+    total_ms = sum(ms)
+    total_ms_max = dist_max(total_ms, world)
+    f_fwd = fwd_flops(w)
+    f_step = 3.5 * f_fwd
+    value = world * f_step * K / (total_ms_max / 1e3) / 1e12
+    bwd_main_avg = sum(main_ms) / K
+    achieved = 2.5 * f_fwd / (bwd_main_avg / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = load_traffic("fa_bwd_main_kernel")
+
+    # end to end through the public API with host buffers: pinned host inputs
+    # copied in, fwd + bwd, gradients copied back, every step
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+        hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v))
+
+        def e2e_step(_):
+            qd.copy_(hq, non_blocking=True)
+            kd.copy_(hk, non_blocking=True)
+            vd.copy_(hv, non_blocking=True)
+            dod.copy_(hdo, non_blocking=True)
+            fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw)
+            fa.fa_bwd(dod, qd, kd, vd, o, lse, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+
+        Ke = max(3, min(K, 20))
+        ems = time_steps(e2e_step, Ke, min(W, 3), lambda: None, stream)
+        e_ms = dist_max(sum(ems), world)
+        h2d = sum(t.numel() * t.element_size() for t in (q, k, v, do))
+        d2h = sum(t.numel() * t.element_size() for t in (dq, dk, dv))
+        e2e = {"value": world * f_step * Ke / (e_ms / 1e3) / 1e12, "unit": "TFLOPS",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
+
+    # per-workload forward table (rank 0, N = 1 only): each pages' config alone
+    table = {}
+    if rank == 0 and world == 1 and not args.no_table:
+        for name in FWD_TABLE:
+            tw = WORKLOADS[name]
+            tq, tk, tv = (t.to(dev) for t in make_workload_inputs(tw, with_dout=False))
+            to = torch.empty_like(tq)
+            tl = torch.empty(tw.batch, tw.q_heads, tw.seqlen_q, dtype=torch.float32, device=dev)
+            tkw = dict(softmax_scale=tw.softmax_scale, causal=tw.causal, window_size=tw.window)
+            tms = time_steps(lambda _: fa.fa_fwd(tq, tk, tv, out=to, lse=tl, **tkw), 20, 3, flush,
+                             stream)
+            med = statistics.median(tms)
+            tf = fwd_flops(tw) / (med / 1e3) / 1e12
+            table[name] = {"fwd_ms_median": round(med, 4), "fwd_ms_min": round(min(tms), 4),
+                           "fwd_tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
+            del tq, tk, tv, to, tl
+        # the main workload's forward and backward separately
+        fms = time_steps(lambda _: fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw), 10, 3, flush,
+                         stream)
+        bms = time_steps(lambda _: fa.fa_bwd(dod, qd, kd, vd, o, lse, dq=dq, dk=dk, dv=dv,
+                                             workspace=ws, **kw), 10, 3, flush, stream)
+        fm, bm = statistics.median(fms), statistics.median(bms)
+        table[w.name] = {"fwd_ms_median": round(fm, 4),
+                         "fwd_tflops": round(f_fwd / (fm / 1e3) / 1e12, 1),
+                         "bwd_ms_median": round(bm, 4),
+                         "bwd_tflops": round(2.5 * f_fwd / (bm / 1e3) / 1e12, 1),
+                         "frac_of_peak_fwd": round(f_fwd / (fm / 1e3) / 1e12 / peak, 4),
+                         "frac_of_peak_bwd": round(2.5 * f_fwd / (bm / 1e3) / 1e12 / peak, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, sample, cores, _, _ = oracle_sample_rate(w, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": round(total_ms_max / K, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q, K, V, dO)",
+            "config": {**w.describe(), "l2": "flushed (256 MB write) before every timed step",
+                       "parallelism": "replicas" if world > 1 else "single GPU",
+                       "step": "fa_fwd + fa_bwd"},
+            "frac_of_peak": round(value / world / peak, 4),
+            "roofline": {"bound": "tensor", "kernel": "fa_bwd_main_kernel",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": "%s bf16_tflops (burst)" % peak_src,
+                         "frac_of_sustained": round(
+                             achieved / float(peaks.get("bf16_tflops_sustained", peak)), 4),
+                         "launch_ms_avg": round(bwd_main_avg, 4)},
+            "clocks": clk,
+            "e2e": e2e,
+            "gpu_launches": 4 * K,
+            "cpu_baseline": cpu,
+            "workloads": table,
+            "wall_s_timed_region": round(t_wall, 3),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The fp64 CPU oracle, as it stands, on bounded samples of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    K, W = args.steps, args.warmup
+    per_step = max(0.5, args.ref_budget_s / max(1, K + W))
+    _, _, cores, T, _ = oracle_sample_rate(w, per_step)
+    import oracle
+    q, k, v, do = make_qkv(1, T, T, 1, 1, w.head_dim, w.dtype, w.seed, with_dout=True)
+    f = lambda t: t.float().double().numpy()  # noqa: E731
+    qq, kk, vv, dd = f(q), f(k), f(v), f(do)
+    flops = 3.5 * 4.0 * w.head_dim * visible_pairs(T, T, w.causal, w.window)
+
+    def step():
+        oracle.attention_fwd(qq, kk, vv, w.softmax_scale, w.causal, w.window)
+        oracle.attention_bwd(qq, kk, vv, dd, w.softmax_scale, w.causal, w.window)
+
+    for _ in range(W):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        step()
+    dt = time.perf_counter() - t0
+    value = flops * K / dt / 1e12
+    sample = ("fp64 oracle fwd+bwd on the first %d tokens of one (batch, head) of %s per step"
+              % (T, w.name))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": K, "warmup": W,
+        "ms_per_step": dt / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) Q, K, V, dO)",
+        "config": {**w.describe(), "sample_tokens": T},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-table", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target duration of the oracle CPU-baseline sample")
+    ap.add_argument("--ref-budget-s", type=float, default=120.0,
+                    help="target duration of the whole reference-arm run")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -35,7 +35,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
-            "fa_get_device_error", "fa_set_wait_limit_ns")
+            "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events")
 
 _lib = None
 
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_get_device_error.restype = i
     lib.fa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.fa_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.fa_set_bwd_main_events.argtypes = [vp, vp]
+    lib.fa_set_bwd_main_events.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -185,6 +187,16 @@ def get_device_error(device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     with torch.cuda.device(dev):
         return int(lib.fa_get_device_error(_stream(dev)))
+
+
+def set_bwd_main_events(start=None, stop=None) -> None:
+    """Have later fa_bwd calls record torch.cuda.Event `start`/`stop` around
+    their main kernel (None, None switches it off).  The events must already
+    exist on the device (record them once before passing them)."""
+    lib = load_library()
+    h0 = ctypes.c_void_p(start.cuda_event) if start is not None else None
+    h1 = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
+    lib.fa_set_bwd_main_events(h0, h1)
 
 
 def set_wait_limit_ns(limit_ns: int) -> int:

@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -19,6 +20,7 @@ namespace {
 __device__ unsigned int g_device_error = 0u;
 
 uint64_t g_wait_limit_ns = 2000000000ull;
+cudaEvent_t g_bwd_ev_start = nullptr, g_bwd_ev_stop = nullptr;
 
 // ------------------------------------------------------------------ driver entry point
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -151,6 +153,23 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <int D, bool BF16>
+int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mdo, const fa::BwdParams& prm, cudaStream_t st) {
+  using Cfg = fa::BwdCfg<D>;
+  auto kern = fa::fa_bwd_main_kernel<D, BF16>;
+  static bool attr_done = false;  // per instantiation and process
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+      return FA_ERR_CUDA;
+    attr_done = true;
+  }
+  dim3 grid(unsigned(prm.B * prm.Hkv), unsigned(prm.n_ntiles));
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mdo, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -166,6 +185,12 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     default: return "unknown status";
   }
+}
+
+int fa_set_bwd_main_events(void* ev_start, void* ev_stop) {
+  g_bwd_ev_start = static_cast<cudaEvent_t>(ev_start);
+  g_bwd_ev_stop = static_cast<cudaEvent_t>(ev_stop);
+  return FA_OK;
 }
 
 uint64_t fa_set_wait_limit_ns(uint64_t limit_ns) {
@@ -228,14 +253,154 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d) {
   if (B < 1 || Nq < 1 || Hq < 1 || d < 1) return 0;
-  return size_t(B) * Nq * Hq * d * sizeof(float) + 2 * size_t(B) * Hq * Nq * sizeof(float) + 256;
+  const size_t nq_pad = (size_t(Nq) + 127) / 128 * 128;
+  return (size_t(B) * Hq * Nq * d + 2 * size_t(B) * Hq * nq_pad) * sizeof(float);
 }
 
-int fa_bwd(const void*, const void*, const void*, const void*, const void*, const float*, void*,
-           void*, void*, void*, size_t, int, int, int, int, int, int, const int64_t*,
-           const int64_t*, const int64_t*, const int64_t*, const int64_t*, const int64_t*,
-           const int64_t*, const int64_t*, int, float, int, int, int, void*) {
-  return FA_ERR_UNSUPPORTED;
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, void* workspace,
+           size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+           const int64_t q_stride[3], const int64_t k_stride[3], const int64_t v_stride[3],
+           const int64_t o_stride[3], const int64_t do_stride[3], const int64_t dq_stride[3],
+           const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
+           float softmax_scale, int causal, int window_left, int window_right, void* stream) {
+  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  if (rc) return rc;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
+      !dk_stride || !dv_stride || !lse)
+    return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdo{dout, do_stride[0], do_stride[1], do_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdq{dq, dq_stride[0], dq_stride[1], dq_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdk{dk, dk_stride[0], dk_stride[1], dk_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tdv{dv, dv_stride[0], dv_stride[1], dv_stride[2], B, Nk, Hkv, d};
+  for (const TensorDesc* t : {&tq, &tk, &tv, &to, &tdo, &tdq, &tdk, &tdv})
+    if ((rc = check_tensor(*t))) return rc;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_ALIGNMENT;
+  const size_t need = fa_bwd_workspace_size(B, Nq, Hq, d);
+  if (workspace == nullptr || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
+  const size_t lse_bytes = size_t(B) * Hq * Nq * sizeof(float);
+  // outputs (dq, dk, dv, workspace) must not overlap each other or any input
+  const TensorDesc* ins[] = {&tq, &tk, &tv, &to, &tdo};
+  const TensorDesc* outs[] = {&tdq, &tdk, &tdv};
+  for (const TensorDesc* ot : outs) {
+    for (const TensorDesc* it : ins)
+      if (overlaps_t(*ot, *it)) return FA_ERR_INVALID_ARG;
+    if (overlaps_span(*ot, lse, lse_bytes) || overlaps_span(*ot, workspace, need))
+      return FA_ERR_INVALID_ARG;
+  }
+  if (overlaps_t(tdq, tdk) || overlaps_t(tdq, tdv) || overlaps_t(tdk, tdv))
+    return FA_ERR_INVALID_ARG;
+  for (const TensorDesc* it : ins)
+    if (overlaps_span(*it, workspace, need)) return FA_ERR_INVALID_ARG;
+  {
+    const uintptr_t w0 = reinterpret_cast<uintptr_t>(workspace);
+    const uintptr_t l0 = reinterpret_cast<uintptr_t>(lse);
+    if (overlaps(w0, w0 + need, l0, l0 + lse_bytes)) return FA_ERR_INVALID_ARG;
+  }
+
+  CUtensorMap mq, mk, mv, mdo;
+  if ((rc = make_map(&mq, tq, dtype)) || (rc = make_map(&mk, tk, dtype)) ||
+      (rc = make_map(&mv, tv, dtype)) || (rc = make_map(&mdo, tdo, dtype)))
+    return rc;
+  unsigned int* err = device_error_ptr();
+  if (!err) return FA_ERR_CUDA;
+  const int nq_pad = (Nq + 127) / 128 * 128;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* lse2 = dq_acc + size_t(B) * Hq * Nq * d;
+  float* Dvec = lse2 + size_t(B) * Hq * nq_pad;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == FA_BF16;
+
+  fa::BwdPrepParams pp{};
+  pp.o = o;
+  pp.dout = dout;
+  pp.lse = lse;
+  pp.lse2 = lse2;
+  pp.Dvec = Dvec;
+  pp.dq_acc = reinterpret_cast<float4*>(dq_acc);
+  pp.o_sb = o_stride[0];
+  pp.o_ss = o_stride[1];
+  pp.o_sh = o_stride[2];
+  pp.do_sb = do_stride[0];
+  pp.do_ss = do_stride[1];
+  pp.do_sh = do_stride[2];
+  pp.B = B;
+  pp.Nq = Nq;
+  pp.Nq_pad = nq_pad;
+  pp.Hq = Hq;
+  pp.d = d;
+  pp.dq_acc_vec4 = int64_t(B) * Hq * Nq * d / 4;
+  {
+    const int64_t rows = int64_t(B) * Hq * nq_pad;
+    const int64_t blocks = std::min<int64_t>((rows + 7) / 8, 148 * 16);
+    if (bf16)
+      fa::fa_bwd_prep_kernel<true><<<unsigned(blocks), 256, 0, st>>>(pp);
+    else
+      fa::fa_bwd_prep_kernel<false><<<unsigned(blocks), 256, 0, st>>>(pp);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+
+  fa::BwdParams bp{};
+  bp.lse2 = lse2;
+  bp.Dvec = Dvec;
+  bp.dq_acc = dq_acc;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.dk_sb = dk_stride[0];
+  bp.dk_ss = dk_stride[1];
+  bp.dk_sh = dk_stride[2];
+  bp.dv_sb = dv_stride[0];
+  bp.dv_ss = dv_stride[1];
+  bp.dv_sh = dv_stride[2];
+  bp.B = B;
+  bp.Nq = Nq;
+  bp.Nq_pad = nq_pad;
+  bp.Nk = Nk;
+  bp.Hq = Hq;
+  bp.Hkv = Hkv;
+  bp.n_ntiles = (Nk + 127) / 128;
+  bp.scale = softmax_scale;
+  bp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  bp.causal = causal ? 1 : 0;
+  bp.wl = window_left;
+  bp.wr = window_right;
+  bp.err = err;
+  bp.wait_limit_ns = g_wait_limit_ns;
+  if (g_bwd_ev_start && cudaEventRecord(g_bwd_ev_start, st) != cudaSuccess) return FA_ERR_CUDA;
+  if (bf16)
+    rc = d == 64 ? launch_bwd<64, true>(mq, mk, mv, mdo, bp, st)
+                 : launch_bwd<128, true>(mq, mk, mv, mdo, bp, st);
+  else
+    rc = d == 64 ? launch_bwd<64, false>(mq, mk, mv, mdo, bp, st)
+                 : launch_bwd<128, false>(mq, mk, mv, mdo, bp, st);
+  if (rc) return rc;
+  if (g_bwd_ev_stop && cudaEventRecord(g_bwd_ev_stop, st) != cudaSuccess) return FA_ERR_CUDA;
+
+  fa::BwdConvertParams cp{};
+  cp.dq_acc = dq_acc;
+  cp.dq = dq;
+  cp.dq_sb = dq_stride[0];
+  cp.dq_ss = dq_stride[1];
+  cp.dq_sh = dq_stride[2];
+  cp.B = B;
+  cp.Nq = Nq;
+  cp.Hq = Hq;
+  cp.d = d;
+  {
+    const int64_t n = int64_t(B) * Hq * Nq * (d / 8);
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 32);
+    if (bf16)
+      fa::fa_bwd_dq_convert_kernel<true><<<unsigned(blocks), 256, 0, st>>>(cp);
+    else
+      fa::fa_bwd_dq_convert_kernel<false><<<unsigned(blocks), 256, 0, st>>>(cp);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 int fa_get_device_error(void* stream) {

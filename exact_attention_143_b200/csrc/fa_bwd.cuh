@@ -1,1 +1,549 @@
+// fa_bwd.cuh -- sm_100a backward kernels of exact attention.
+//
+// The backward recomputes the probabilities from the forward's per-row
+// log-sum-exp instead of storing them ("tiling and recomputation",
+// "optimizing-attention-flash", Quick start; "Что такое FlashAttention…",
+// section "Основной механизм простыми словами": tiling and recomputation).
+// With P = exp(scale * Q K^T - LSE) on visible keys, the gradient of
+// L = sum(dO * O) is the textbook one:
+//   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),
+//   dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three launches:
+//   1. fa_bwd_prep_kernel: D_i = sum_c dO_ic O_ic and LSE2_i = LSE_i * log2(e)
+//      (fp32, padded to a multiple of 128 rows), and zeroes the fp32 dQ
+//      accumulator.
+//   2. fa_bwd_main_kernel: one CTA per (128-key tile, kv head, batch).  K and V
+//      stay in shared memory; the CTA loops over every query tile that can see
+//      its keys, for every query head of the GQA group, so dK and dV are summed
+//      in tensor memory without atomics.  Per step (query tile i, head h):
+//        S^T  = K Q_i^T        (tcgen05, A = K, B = Q_i, both from smem)
+//        dP^T = V dO_i^T       (A = V, B = dO_i)
+//        P^T  = exp2(S^T * scale * log2 e - LSE2)   (compute warps, written
+//                                                    back as 16-bit over S^T)
+//        dV  += P^T dO_i       (A = P^T from tensor memory)
+//        dS^T = P^T * (dP^T - D)                     (to tensor memory and to
+//                                                    smem as the dQ operand)
+//        dK  += dS^T Q_i       (A = dS^T from tensor memory)
+//        dQ_i = dS K           (A = dS from smem, MN-major)
+//      and the dQ warps add scale * dQ_i into the fp32 accumulator.
+//   3. fa_bwd_dq_convert_kernel: dQ accumulator -> dQ in the input dtype.
+//
+// Roles (320 threads): warps 0-3 compute (thread = key row = tensor-memory
+// lane), warps 4-7 dQ readout (thread = query row), warp 8 MMA issuer,
+// warp 9 TMA producer.  Tensor memory: two 128-column regions R0/R1 swap
+// roles every step (S/P/dQ in one, dP/dS in the other), dK at 256, dV at
+// 256 + d.
 #pragma once
+
+#include <climits>
+
+#include <cuda_fp16.h>
+
+#include "fa_ptx.cuh"
+
+namespace fa {
+
+// ------------------------------------------------------------------ kernel 1
+struct BwdPrepParams {
+  const void* o;
+  const void* dout;
+  const float* lse;
+  float* lse2;     // [B, Hq, Nq_pad]
+  float* Dvec;     // [B, Hq, Nq_pad]
+  float4* dq_acc;  // [B, Hq, Nq, d] fp32, zeroed here
+  int64_t o_sb, o_ss, o_sh, do_sb, do_ss, do_sh;
+  int B, Nq, Nq_pad, Hq, d;
+  int64_t dq_acc_vec4;  // number of float4 in dq_acc
+};
+
+template <bool BF16>
+__device__ __forceinline__ float to_f32(uint16_t x) {
+  if constexpr (BF16) {
+    return __uint_as_float(uint32_t(x) << 16);
+  } else {
+    return __half2float(__ushort_as_half(x));
+  }
+}
+
+// One warp per (b, h, row); lane l handles elements l, l+32, ... of head_dim.
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p) {
+  const int64_t nrows = int64_t(p.B) * p.Hq * p.Nq_pad;
+  const int64_t warp_id = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = warp_id; r < nrows; r += nwarps) {
+    const int i = int(r % p.Nq_pad);
+    const int64_t bh = r / p.Nq_pad;
+    const int h = int(bh % p.Hq), b = int(bh / p.Hq);
+    float acc = 0.f, lse2 = INFINITY;
+    if (i < p.Nq) {
+      const uint16_t* orow = static_cast<const uint16_t*>(p.o) + b * p.o_sb + int64_t(i) * p.o_ss +
+                             int64_t(h) * p.o_sh;
+      const uint16_t* drow = static_cast<const uint16_t*>(p.dout) + b * p.do_sb +
+                             int64_t(i) * p.do_ss + int64_t(h) * p.do_sh;
+      for (int c = lane; c < p.d; c += 32) acc += to_f32<BF16>(orow[c]) * to_f32<BF16>(drow[c]);
+      const float l = p.lse[(int64_t(b) * p.Hq + h) * p.Nq + i];
+      lse2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      p.Dvec[r] = acc;
+      p.lse2[r] = lse2;
+    }
+  }
+  // zero the dQ accumulator
+  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t x = tid; x < p.dq_acc_vec4; x += nthr) p.dq_acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ------------------------------------------------------------------ kernel 3
+struct BwdConvertParams {
+  const float* dq_acc;  // [B, Hq, Nq, d]
+  void* dq;
+  int64_t dq_sb, dq_ss, dq_sh;
+  int B, Nq, Hq, d;
+};
+
+// One thread per 8 consecutive elements of one row (16-byte store).
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdConvertParams p) {
+  const int per_row = p.d / 8;
+  const int64_t n = int64_t(p.B) * p.Hq * p.Nq * per_row;
+  for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < n;
+       x += int64_t(gridDim.x) * blockDim.x) {
+    const int c8 = int(x % per_row);
+    const int64_t row = x / per_row;  // (b, h, i)
+    const int i = int(row % p.Nq);
+    const int64_t bh = row / p.Nq;
+    const int h = int(bh % p.Hq), b = int(bh / p.Hq);
+    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + row * p.d + c8 * 8);
+    const float4 a = src[0], c = src[1];
+    uint4 out;
+    out.x = pack2<BF16>(a.x, a.y);
+    out.y = pack2<BF16>(a.z, a.w);
+    out.z = pack2<BF16>(c.x, c.y);
+    out.w = pack2<BF16>(c.z, c.w);
+    uint16_t* dst = static_cast<uint16_t*>(p.dq) + b * p.dq_sb + int64_t(i) * p.dq_ss +
+                    int64_t(h) * p.dq_sh + c8 * 8;
+    *reinterpret_cast<uint4*>(dst) = out;
+  }
+}
+
+// ------------------------------------------------------------------ kernel 2
+struct BwdParams {
+  const float* lse2;  // [B, Hq, Nq_pad]
+  const float* Dvec;  // [B, Hq, Nq_pad]
+  float* dq_acc;      // [B, Hq, Nq, d]
+  void* dk;
+  void* dv;
+  int64_t dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
+  int B, Nq, Nq_pad, Nk, Hq, Hkv;
+  int n_ntiles;     // ceil(Nk / 128)
+  float scale;      // softmax_scale (signed)
+  float scale_log2; // softmax_scale * log2(e) (signed)
+  int causal, wl, wr;
+  unsigned int* err;
+  uint64_t wait_limit_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kChunk = 128 * 64 * 2;     // 128 rows x 64 columns, 16-bit, swizzled
+  static constexpr int kTileBytes = 128 * D * 2;  // a 128-row tile
+  static constexpr int kThreads = 320;
+  static constexpr int kSmemK = 0;
+  static constexpr int kSmemV = kSmemK + kTileBytes;
+  static constexpr int kSmemQ = kSmemV + kTileBytes;        // 2 stages
+  static constexpr int kSmemDO = kSmemQ + 2 * kTileBytes;   // 2 stages
+  static constexpr int kSmemDS = kSmemDO + 2 * kTileBytes;  // 128 keys x 128 queries, 16-bit
+  static constexpr int kSmemLSE = kSmemDS + 2 * kChunk;     // 2 stages x 128 fp32
+  static constexpr int kSmemDv = kSmemLSE + 2 * 512;        // 2 stages x 128 fp32
+  static constexpr int kSmemBar = kSmemDv + 2 * 512;
+  static constexpr int kSmemBytes = kSmemBar + 256;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColDK = 256;
+  static constexpr uint32_t kColDV = 256 + D;
+};
+
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
+                                             uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(320, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(p.err, kDevErrTimeout);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kSmemBar);
+  const uint32_t bar_kv = smem_u32(&bars[0]);
+  auto bar_qfull = [&](int st) { return smem_u32(&bars[1 + st]); };
+  auto bar_qempty = [&](int st) { return smem_u32(&bars[3 + st]); };
+  const uint32_t bar_s = smem_u32(&bars[5]);
+  const uint32_t bar_dp = smem_u32(&bars[6]);
+  const uint32_t bar_p = smem_u32(&bars[7]);
+  const uint32_t bar_ds = smem_u32(&bars[8]);
+  const uint32_t bar_dq = smem_u32(&bars[9]);
+  const uint32_t bar_dqfree = smem_u32(&bars[10]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kSmemBar + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kSmemBar + 136);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // work unit: (batch, kv head) from blockIdx.x, key tile from blockIdx.y
+  const int bg = blockIdx.x;
+  const int g = bg % p.Hkv;
+  const int b = bg / p.Hkv;
+  const int ntile = int(blockIdx.y);
+  const int G = p.Hq / p.Hkv;
+  const int key0 = ntile * 128;
+
+  // query rows that can see some key of this tile (bounds are monotone in the row)
+  const int off = p.Nk - p.Nq;
+  const int right = p.causal ? 0 : p.wr;
+  const int key1 = min(key0 + 127, p.Nk - 1);
+  int i_min = right >= 0 ? max(0, key0 - off - right) : 0;
+  int i_max = p.wl >= 0 ? min(p.Nq - 1, key1 - off + p.wl) : p.Nq - 1;
+  const int mlo = i_min / 128;
+  const int nm = (i_min <= i_max) ? (i_max / 128 - mlo + 1) : 0;
+  const int T = nm * G;  // steps: (query head, query tile)
+
+  WaitCtx wc{abort_flag, p.err, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(bar_qfull(st), 1);
+      mbar_init(bar_qempty(st), 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 128);
+    mbar_init(bar_ds, 128);
+    mbar_init(bar_dq, 1);
+    mbar_init(bar_dqfree, 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  __syncwarp();
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto step_head = [&](int s) { return g * G + s / nm; };
+  auto step_mtile = [&](int s) { return mlo + s % nm; };
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && T > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar_kv, 2 * Cfg::kTileBytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(sbase + Cfg::kSmemK + c * Cfg::kChunk, &tmK, bar_kv, c * 64, key0, g, b);
+        tma_load_4d(sbase + Cfg::kSmemV + c * Cfg::kChunk, &tmV, bar_kv, c * 64, key0, g, b);
+      }
+      for (int s = 0; s < T; ++s) {
+        const int st = s & 1, u = s >> 1;
+        if (u > 0 && !mbar_wait(bar_qempty(st), (u - 1) & 1, wc)) break;
+        const int h = step_head(s), m = step_mtile(s);
+        mbar_arrive_expect_tx(bar_qfull(st), 2 * Cfg::kTileBytes + 1024);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(sbase + Cfg::kSmemQ + st * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ,
+                      bar_qfull(st), c * 64, m * 128, h, b);
+          tma_load_4d(sbase + Cfg::kSmemDO + st * Cfg::kTileBytes + c * Cfg::kChunk, &tmDO,
+                      bar_qfull(st), c * 64, m * 128, h, b);
+        }
+        const int64_t rowoff = (int64_t(b) * p.Hq + h) * p.Nq_pad + int64_t(m) * 128;
+        bulk_load_1d(sbase + Cfg::kSmemLSE + st * 512, p.lse2 + rowoff, 512, bar_qfull(st));
+        bulk_load_1d(sbase + Cfg::kSmemDv + st * 512, p.Dvec + rowoff, 512, bar_qfull(st));
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      const uint32_t idesc_ss = make_idesc_f16(BF16, 128, 128, false, false);   // S^T, dP^T
+      const uint32_t idesc_acc = make_idesc_f16(BF16, 128, D, false, true);    // dV, dK
+      const uint32_t idesc_dq = make_idesc_f16(BF16, 128, D, true, true);      // dQ
+      const uint32_t sK = sbase + Cfg::kSmemK, sV = sbase + Cfg::kSmemV;
+      const uint32_t sDS = sbase + Cfg::kSmemDS;
+      bool ok = mbar_wait(bar_kv, 0, wc);
+      for (int s = 0; s < T && ok; ++s) {
+        const int st = s & 1, u = s >> 1;
+        const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
+        const uint32_t sQ = sbase + Cfg::kSmemQ + st * Cfg::kTileBytes;
+        const uint32_t sDO = sbase + Cfg::kSmemDO + st * Cfg::kTileBytes;
+        if (!(ok = mbar_wait(bar_qfull(st), u & 1, wc))) break;
+        tc_fence_after();
+        // S^T = K Q^T (M = keys, N = queries, K-dim = d)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * Cfg::kChunk + (kk & 3) * 32;
+          mma_ss(Ra, make_sdesc_sw128(sK + o, 16, 1024), make_sdesc_sw128(sQ + o, 16, 1024),
+                 idesc_ss, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s);
+        // dP^T = V dO^T, into the region the previous dQ used
+        if (s > 0 && !(ok = mbar_wait(bar_dqfree, (s - 1) & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * Cfg::kChunk + (kk & 3) * 32;
+          mma_ss(Rb, make_sdesc_sw128(sV + o, 16, 1024), make_sdesc_sw128(sDO + o, 16, 1024),
+                 idesc_ss, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_dp);
+        // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major)
+        if (!(ok = mbar_wait(bar_p, s & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + Cfg::kColDV, Ra + kk * 8,
+                 make_sdesc_sw128(sDO + kk * 2048, Cfg::kChunk, 1024), idesc_acc,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q ; dQ = dS K
+        if (!(ok = mbar_wait(bar_ds, s & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + Cfg::kColDK, Rb + kk * 8,
+                 make_sdesc_sw128(sQ + kk * 2048, Cfg::kChunk, 1024), idesc_acc,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(Ra, make_sdesc_sw128(sDS + kk * 2048, Cfg::kChunk, 1024),
+                 make_sdesc_sw128(sK + kk * 2048, Cfg::kChunk, 1024), idesc_dq,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar_dq);
+        mma_commit(bar_qempty(st));
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute: P^T, dS^T
+    const int j = threadIdx.x;  // key row within the tile == tensor-memory lane
+    const int key = key0 + j;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    // queries that see this key: [qlo, qhi]
+    int qlo = right >= 0 ? key - off - right : INT_MIN;
+    int qhi = p.wl >= 0 ? key - off + p.wl : INT_MAX;
+    if (key >= p.Nk) {
+      qlo = INT_MAX;
+      qhi = INT_MIN;
+    }
+    const float sc = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < T; ++s) {
+      const int st = s & 1;
+      const uint32_t Ra = tmem + lane_base + (s & 1) * 128;
+      const uint32_t Rb = tmem + lane_base + ((s + 1) & 1) * 128;
+      const float* lse2 = reinterpret_cast<const float*>(smem + Cfg::kSmemLSE + st * 512);
+      const float* Dv = reinterpret_cast<const float*>(smem + Cfg::kSmemDv + st * 512);
+      const int q0 = step_mtile(s) * 128;
+      const bool need_mask = __any_sync(0xffffffffu, qlo > q0 || qhi < q0 + 127);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s, s & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      // P^T = exp2(S^T * scale * log2 e - LSE2), 32 queries at a time
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t sr[32];
+        tmem_ld32(Ra + c0, sr);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
+          float pv[4];
+          pv[0] = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, -l4.x));
+          pv[1] = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, -l4.y));
+          pv[2] = fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sc, -l4.z));
+          pv[3] = fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sc, -l4.w));
+          if (need_mask) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = q0 + c0 + c + e;
+              pv[e] = (q >= qlo && q <= qhi) ? pv[e] : 0.f;
+            }
+          }
+          pk[c / 2] = pack2<BF16>(pv[0], pv[1]);
+          pk[c / 2 + 1] = pack2<BF16>(pv[2], pv[3]);
+        }
+        // P^T packed: 32 queries -> 16 columns, written over columns already read
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(Ra + c0 / 2),
+            "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+            "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
+            "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+            : "memory");
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+      // dS^T = P^T * (dP^T - D); the smem copy waits until the previous dQ MMA is done
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, s & 1, wc));
+      if (ok && s > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (s - 1) & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint8_t* dsrow = smem + Cfg::kSmemDS + j * 128;
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t dpr[32], pr[16];
+        tmem_ld32(Rb + c0, dpr);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(pr[0]), "=r"(pr[1]), "=r"(pr[2]), "=r"(pr[3]), "=r"(pr[4]), "=r"(pr[5]),
+              "=r"(pr[6]), "=r"(pr[7]), "=r"(pr[8]), "=r"(pr[9]), "=r"(pr[10]), "=r"(pr[11]),
+              "=r"(pr[12]), "=r"(pr[13]), "=r"(pr[14]), "=r"(pr[15])
+            : "r"(Ra + c0 / 2));
+        tmem_wait_ld();
+        uint32_t dk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(Dv + c0 + c);
+          float pf[4];
+          if constexpr (BF16) {
+            pf[0] = __uint_as_float(pr[c / 2] << 16);
+            pf[1] = __uint_as_float(pr[c / 2] & 0xFFFF0000u);
+            pf[2] = __uint_as_float(pr[c / 2 + 1] << 16);
+            pf[3] = __uint_as_float(pr[c / 2 + 1] & 0xFFFF0000u);
+          } else {
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&pr[c / 2]));
+            const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&pr[c / 2 + 1]));
+            pf[0] = a.x;
+            pf[1] = a.y;
+            pf[2] = bb.x;
+            pf[3] = bb.y;
+          }
+          const float ds0 = pf[0] * (__uint_as_float(dpr[c]) - d4.x);
+          const float ds1 = pf[1] * (__uint_as_float(dpr[c + 1]) - d4.y);
+          const float ds2 = pf[2] * (__uint_as_float(dpr[c + 2]) - d4.z);
+          const float ds3 = pf[3] * (__uint_as_float(dpr[c + 3]) - d4.w);
+          dk[c / 2] = pack2<BF16>(ds0, ds1);
+          dk[c / 2 + 1] = pack2<BF16>(ds2, ds3);
+        }
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(Rb + c0 / 2),
+            "r"(dk[0]), "r"(dk[1]), "r"(dk[2]), "r"(dk[3]), "r"(dk[4]), "r"(dk[5]), "r"(dk[6]),
+            "r"(dk[7]), "r"(dk[8]), "r"(dk[9]), "r"(dk[10]), "r"(dk[11]), "r"(dk[12]),
+            "r"(dk[13]), "r"(dk[14]), "r"(dk[15])
+            : "memory");
+        // smem copy in the MN-major 128-byte-swizzled layout of the dQ A operand:
+        // chunk (c0 / 64) holds queries [64 chunk, +64) of every key row; the
+        // 16-byte unit u of row j sits at unit u ^ (j % 8).
+        uint8_t* chunk = dsrow + (c0 >> 6) * Cfg::kChunk;
+        const int u0 = (c0 & 63) >> 3;  // first 16-byte unit of these 32 queries
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          const int u = (u0 + uu) ^ (j & 7);
+          *reinterpret_cast<uint4*>(chunk + u * 16) =
+              make_uint4(dk[4 * uu], dk[4 * uu + 1], dk[4 * uu + 2], dk[4 * uu + 3]);
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+    }
+    // epilogue: dK = scale * (dS^T Q summed), dV = (P^T dO summed), in the input dtype
+    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (T - 1) & 1, wc));
+    if (ok) {
+      tc_fence_after();
+      const bool store = key < p.Nk;
+      uint16_t* dkrow = static_cast<uint16_t*>(p.dk) + b * p.dk_sb + int64_t(key) * p.dk_ss +
+                        int64_t(g) * p.dk_sh;
+      uint16_t* dvrow = static_cast<uint16_t*>(p.dv) + b * p.dv_sb + int64_t(key) * p.dv_ss +
+                        int64_t(g) * p.dv_sh;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? Cfg::kColDK : Cfg::kColDV;
+        const float mul = which == 0 ? p.scale : 1.f;
+        uint16_t* dst_row = which == 0 ? dkrow : dvrow;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          if (T > 0) {
+            tmem_ld32(tmem + lane_base + col + c0, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = 0u;
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pkd[c] = pack2<BF16>(__uint_as_float(r[2 * c]) * mul,
+                                 __uint_as_float(r[2 * c + 1]) * mul);
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c0);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              dst[q4] = make_uint4(pkd[4 * q4], pkd[4 * q4 + 1], pkd[4 * q4 + 2], pkd[4 * q4 + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ readout (warps 4-7)
+    const int r = threadIdx.x - 128;  // query row within the tile == tensor-memory lane
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    for (int s = 0; s < T; ++s) {
+      const uint32_t Ra = tmem + lane_base + (s & 1) * 128;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, s & 1, wc))) break;
+      tc_fence_after();
+      uint32_t v[D];
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(Ra + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_dqfree);
+      const int h = step_head(s), row = step_mtile(s) * 128 + r;
+      if (row < p.Nq) {
+        float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((int64_t(b) * p.Hq + h) * p.Nq + row) * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c)
+          atomicAdd(dst + c, make_float4(__uint_as_float(v[4 * c]) * p.scale,
+                                         __uint_as_float(v[4 * c + 1]) * p.scale,
+                                         __uint_as_float(v[4 * c + 2]) * p.scale,
+                                         __uint_as_float(v[4 * c + 3]) * p.scale));
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -131,6 +131,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
 int fa_get_device_error(void* stream);
 
 /*
+ * Optional instrumentation.  When ev_start and ev_stop are cudaEvent_t
+ * handles (passed as void pointers), every later fa_bwd call records
+ * ev_start on its stream right before it launches its main kernel and
+ * ev_stop right after, so the caller can time that kernel alone with
+ * cudaEventElapsedTime.  NULL, NULL turns it off.  The caller owns the
+ * events; the setting is process-wide.  Returns FA_OK.
+ */
+int fa_set_bwd_main_events(void* ev_start, void* ev_stop);
+
+/*
  * Sets the per-wait limit of device-side waits, in nanoseconds (default
  * 2e9).  Returns the previous value.  For tests of the timeout path only.
  */
