@@ -35,7 +35,8 @@ FA_ERR_DEVICE_TIMEOUT = 6
 
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
-            "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events")
+            "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
+            "fa_bwd_noalloc")
 
 _lib = None
 
@@ -72,6 +73,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_set_wait_limit_ns.restype = ctypes.c_uint64
     lib.fa_set_bwd_main_events.argtypes = [vp, vp]
     lib.fa_set_bwd_main_events.restype = i
+    lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [i64p] * 8 + [i, f, i, i, i, vp]
+    lib.fa_bwd_noalloc.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib

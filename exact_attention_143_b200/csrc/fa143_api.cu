@@ -414,3 +414,53 @@ int fa_get_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation backward
+// fa_bwd_noalloc: the backward for callers that cannot call cudaMalloc.  Its
+// scratch is this file-scope device array; host code must not pass the
+// array's name to a kernel (in host code it is only a stand-in), so the
+// device address is looked up once per device with cudaGetSymbolAddress.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device (looked up on the
+// first call per device), or nullptr on failure.
+void* noalloc_scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = p;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                              const int64_t q_stride[3], const int64_t k_stride[3],
+                              const int64_t v_stride[3], const int64_t o_stride[3],
+                              const int64_t do_stride[3], const int64_t dq_stride[3],
+                              const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
+                              float softmax_scale, int causal, int window_left,
+                              int window_right, void* stream) {
+  const size_t need = fa_bwd_workspace_size(B, Nq, Hq, d);
+  if (need > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;  // larger than the array
+  void* scratch = noalloc_scratch_address();
+  if (scratch == nullptr) return FA_ERR_CUDA;
+  // fa_bwd zeroes the dQ accumulator and rewrites the row terms on every call,
+  // so the previous call's contents of the shared array do not matter.
+  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, Nq,
+                Nk, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride,
+                dk_stride, dv_stride, dtype, softmax_scale, causal, window_left, window_right,
+                stream);
+}

@@ -124,6 +124,41 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            int window_right, void* stream);
 
 /*
+ * Backward pass for callers that cannot allocate device memory.
+ *
+ * Some callers of this library cannot call cudaMalloc: for example a plugin
+ * running inside a host framework that owns all device memory and gives
+ * its operators no workspace, or a latency-critical loop where an
+ * allocation's implicit device synchronisation is not allowed.  This entry
+ * point takes the same arguments as fa_bwd minus the workspace, and uses a
+ * scratch buffer built into the library instead: a static device array of
+ * FA_BWD_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library
+ * holds until the process exits.  It allocates nothing itself.
+ *
+ *  - Sizes whose fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_SCRATCH_BYTES
+ *    are rejected with FA_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device looks up the buffer's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one buffer, which keeps the previous call's
+ *    contents (the kernels re-initialise what must start at zero).  Calls
+ *    that overlap on the GPU (for example on two streams at once) race on it.
+ * Results equal fa_bwd's (dQ up to the order of its fp32 atomic adds).
+ * The pages describe no such variant; it has no counterpart there.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                   int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                   const int64_t q_stride[3], const int64_t k_stride[3],
+                   const int64_t v_stride[3], const int64_t o_stride[3],
+                   const int64_t do_stride[3], const int64_t dq_stride[3],
+                   const int64_t dk_stride[3], const int64_t dv_stride[3],
+                   int dtype, float softmax_scale, int causal, int window_left,
+                   int window_right, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device error word of
  * the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel gave up
  * on a bounded wait since the last call (FA_ERR_CUDA if the query failed).
