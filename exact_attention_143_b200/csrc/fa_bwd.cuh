@@ -286,61 +286,82 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && T > 0) {
+    // The whole warp runs this loop and waits; one elected lane issues each
+    // batch of MMAs and its commits.
+    if (T > 0) {
       const uint32_t idesc_ss = make_idesc_f16(BF16, 128, 128, false, false);   // S^T, dP^T
       const uint32_t idesc_acc = make_idesc_f16(BF16, 128, D, false, true);    // dV, dK
       const uint32_t idesc_dq = make_idesc_f16(BF16, 128, D, true, true);      // dQ
-      const uint32_t sK = sbase + Cfg::kSmemK, sV = sbase + Cfg::kSmemV;
-      const uint32_t sDS = sbase + Cfg::kSmemDS;
-      bool ok = mbar_wait(bar_kv, 0, wc);
+      auto wait_all = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+      };
+      // descriptors are built once; an MMA only adds a compile-time offset
+      constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
+      constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // MN-major tiles
+      const uint64_t dK_k = sdesc_at(kDescK, sbase + Cfg::kSmemK);
+      const uint64_t dV_k = sdesc_at(kDescK, sbase + Cfg::kSmemV);
+      const uint64_t dK_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemK);
+      const uint64_t dDS_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDS);
+      const uint64_t dQ_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
+      const uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
+      const uint64_t dDO_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
+      const uint64_t dDO_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
+      bool ok = wait_all(bar_kv, 0);
       for (int s = 0; s < T && ok; ++s) {
         const int st = s & 1, u = s >> 1;
         const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
-        const uint32_t sQ = sbase + Cfg::kSmemQ + st * Cfg::kTileBytes;
-        const uint32_t sDO = sbase + Cfg::kSmemDO + st * Cfg::kTileBytes;
-        if (!(ok = mbar_wait(bar_qfull(st), u & 1, wc))) break;
+        const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
+        if (!(ok = wait_all(bar_qfull(st), u & 1))) break;
         tc_fence_after();
         // S^T = K Q^T (M = keys, N = queries, K-dim = d)
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * Cfg::kChunk + (kk & 3) * 32;
-          mma_ss(Ra, make_sdesc_sw128(sK + o, 16, 1024), make_sdesc_sw128(sQ + o, 16, 1024),
-                 idesc_ss, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+            mma_ss(Ra, dK_k + o, dQ_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_s);
         }
-        mma_commit(bar_s);
+        __syncwarp();
         // dP^T = V dO^T, into the region the previous dQ used
-        if (s > 0 && !(ok = mbar_wait(bar_dqfree, (s - 1) & 1, wc))) break;
+        if (s > 0 && !(ok = wait_all(bar_dqfree, (s - 1) & 1))) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * Cfg::kChunk + (kk & 3) * 32;
-          mma_ss(Rb, make_sdesc_sw128(sV + o, 16, 1024), make_sdesc_sw128(sDO + o, 16, 1024),
-                 idesc_ss, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+            mma_ss(Rb, dV_k + o, dDO_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_dp);
         }
-        mma_commit(bar_dp);
+        __syncwarp();
         // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major)
-        if (!(ok = mbar_wait(bar_p, s & 1, wc))) break;
+        if (!(ok = wait_all(bar_p, s & 1))) break;
         tc_fence_after();
+        const uint32_t acc0 = s > 0 ? 1u : 0u;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + Cfg::kColDV, Ra + kk * 8,
-                 make_sdesc_sw128(sDO + kk * 2048, Cfg::kChunk, 1024), idesc_acc,
-                 (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + Cfg::kColDV, Ra + kk * 8,
+                   dDO_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
+        }
+        __syncwarp();
         // dK += dS^T Q ; dQ = dS K
-        if (!(ok = mbar_wait(bar_ds, s & 1, wc))) break;
+        if (!(ok = wait_all(bar_ds, s & 1))) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + Cfg::kColDK, Rb + kk * 8,
-                 make_sdesc_sw128(sQ + kk * 2048, Cfg::kChunk, 1024), idesc_acc,
-                 (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + Cfg::kColDK, Rb + kk * 8,
+                   dQ_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(Ra, make_sdesc_sw128(sDS + kk * 2048, Cfg::kChunk, 1024),
-                 make_sdesc_sw128(sK + kk * 2048, Cfg::kChunk, 1024), idesc_dq,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq);
-        mma_commit(bar_qempty(st));
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(Ra, dDS_mn + uint64_t((kk * 2048) >> 4), dK_mn + uint64_t((kk * 2048) >> 4),
+                   idesc_dq, kk > 0 ? 1u : 0u);
+          mma_commit(bar_dq);
+          mma_commit(bar_qempty(st));
+        }
+        __syncwarp();
       }
     }
   } else if (warp < 4) {

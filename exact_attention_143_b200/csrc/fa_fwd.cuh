@@ -17,12 +17,18 @@
 //   warps 0-3/4-7 softmax warpgroup of tile 0/1: thread r owns row r of its
 //                tile (tensor-memory lane r), so row max and row sum are
 //                in-thread; it masks boundary tiles, keeps the running max m
-//                and sum l, writes P (16-bit) back over S, rescales O in
+//                and sum l, writes P (16-bit) to tensor memory, rescales O in
 //                tensor memory when m grows by more than 2^8 (exact: the
 //                final O / l uses the same m), and runs the epilogue
 //                (O / l to HBM, LSE = ln 2 * (m + log2 l)).
-// Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 at
-// 256 and 256 + d.  K/V tiles that no row of a tile can see are skipped whole.
+// Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 at 256
+// and 256 + d.  With d = 64 the 128 spare columns hold P_0 and P_1, so
+// S_t(j+1) is computed while the softmax of S_t(j) is still running; with
+// d = 128 P_t is written over S_t and S_t(j+1) waits for P_t V_j.
+// The exponentials are split between the MUFU unit (ex2.approx) and a
+// polynomial on the FMA pipe (fit by fit_exp2_poly.py), which keeps the
+// special-function unit from bounding the kernel.  K/V tiles that no row of
+// a tile can see are skipped whole.
 #pragma once
 
 #include "fa_ptx.cuh"
@@ -44,9 +50,7 @@ struct FwdParams {
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kRows = 128;                 // rows per query tile (MMA M)
-  static constexpr int kTiles = 2;                  // query tiles per CTA
-  static constexpr int kKeys = 128;                 // keys per K/V tile (MMA N of Q K^T)
+  static constexpr int kTiles = 2;                  // query tiles of 128 rows per CTA
   static constexpr int kChunk = 128 * 64 * 2;       // one 128-row x 64-column swizzled chunk
   static constexpr int kTileBytes = 128 * D * 2;    // a 128-row tile
   static constexpr int kStages = D == 64 ? 4 : 2;   // K ring and V ring depth
@@ -57,6 +61,10 @@ struct FwdCfg {
   static constexpr int kSmemBytes = kSmemV + kStages * kTileBytes + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
+  static constexpr bool kSepP = D == 64;            // P in its own tensor-memory region
+  static constexpr uint32_t kColP = 384;            // P_t at 384 + 64 t (d = 64 only)
+  // of every 8 column pairs of a row, how many take the FMA-pipe exp2
+  static constexpr int kEmuPairsPer8 = D == 64 ? 3 : 1;
 };
 
 // Visible key range of query row i, [lo, hi] inclusive; empty if lo > hi.
@@ -68,12 +76,54 @@ __device__ __forceinline__ void row_key_range(int i, int Nq, int Nk, int causal,
   hi = right >= 0 ? min(Nk - 1, ip + right) : Nk - 1;
 }
 
+// ---------------------------------------------------------------- exp2 on the FMA pipe
+// 2^x for a pair: x = n + f with n = round(x) (the 1.5 * 2^23 addition rounds
+// to an integer in the low mantissa bits), f in [-1/2, 1/2]; 2^f by a minimax
+// polynomial (relative error 2.7e-6 at degree 4, 7.5e-5 at degree 3, see
+// fit_exp2_poly.py); 2^n built directly in the exponent field.  x is clamped
+// at -127 first, where the exponent field becomes 0 and the result is +0, so
+// masked (-inf) scores give exactly 0.
+template <bool BF16>
+__device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p;
+  if constexpr (BF16) {  // degree 3: far below bf16 rounding of P
+    p = __ffma2_rn(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
+                   make_float2(2.426111251e-01f, 2.426111251e-01f));
+    p = __ffma2_rn(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+    p = __ffma2_rn(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+  } else {  // degree 4: below fp16 rounding of P
+    p = __ffma2_rn(make_float2(9.570102207e-03f, 9.570102207e-03f), f,
+                   make_float2(5.591785908e-02f, 5.591785908e-02f));
+    p = __ffma2_rn(p, f, make_float2(2.402474433e-01f, 2.402474433e-01f));
+    p = __ffma2_rn(p, f, make_float2(6.931217909e-01f, 6.931217909e-01f));
+    p = __ffma2_rn(p, f, make_float2(9.999992847e-01f, 9.999992847e-01f));
+  }
+  // (n + 127) << 23: the low bits of t hold n + 2^22 + 2^23, whose shifted-out
+  // high part vanishes modulo 2^32
+  const float sx = __uint_as_float((__float_as_uint(t.x) << 23) + (127u << 23));
+  const float sy = __uint_as_float((__float_as_uint(t.y) << 23) + (127u << 23));
+  return __fmul2_rn(p, make_float2(sx, sy));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(320, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int S = Cfg::kStages;
+  constexpr bool kSepP = Cfg::kSepP;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms.
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -90,13 +140,15 @@ __global__ void __launch_bounds__(320, 1)
   auto bar_sfull = [&](int t) { return smem_u32(&bars[1 + 4 * S + t]); };
   auto bar_pfull = [&](int t) { return smem_u32(&bars[3 + 4 * S + t]); };
   auto bar_odone = [&](int t) { return smem_u32(&bars[5 + 4 * S + t]); };
+  auto bar_sfree = [&](int t) { return smem_u32(&bars[7 + 4 * S + t]); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // work unit: (batch, head) from blockIdx.x, heaviest query block first
+  // work unit: (batch, head) from blockIdx.x, query block from blockIdx.y with
+  // the heaviest (latest, under a causal mask) blocks launched first
   const int bh = blockIdx.x;
   const int h = bh % p.Hq;
   const int b = bh / p.Hq;
@@ -140,6 +192,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar_sfull(t), 1);
       mbar_init(bar_pfull(t), 128);
       mbar_init(bar_odone(t), 1);
+      mbar_init(bar_sfree(t), 128);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -185,58 +238,110 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && JHI > JLO) {
+    // The whole warp runs this loop and waits; one elected lane issues each
+    // batch of MMAs and its commit.
+    if (JHI > JLO) {
       const uint32_t idesc_qk = make_idesc_f16(BF16, 128, 128, false, false) | (p.qk_negate << 13);
       const uint32_t idesc_pv = make_idesc_f16(BF16, 128, D, false, true);
-      bool ok = mbar_wait(bar_q, 0, wc);
+      auto wait_all = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+      };
+      bool ok = wait_all(bar_q, 0);
       auto in_range = [&](int t, int j) {
         return t ? (j >= jlo1 && j < jhi1) : (j >= jlo0 && j < jhi0);
       };
+      // descriptors are built once; an MMA only adds a compile-time offset
+      // (address >> 4) to them
+      constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
+      constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // V, MN-major
+      const uint64_t dQ0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
+      const uint64_t dK0 = sdesc_at(kDescK, sbase + Cfg::kSmemK);
+      const uint64_t dV0 = sdesc_at(kDescMN, sbase + Cfg::kSmemV);
       auto issue_s = [&](int t, int j) -> bool {
         const int idx = j - JLO, s = idx % S, u = idx / S;
-        if (!mbar_wait(bar_kfull(s), u & 1, wc)) return false;
+        if (!wait_all(bar_kfull(s), u & 1)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + Cfg::kSmemQ + t * Cfg::kTileBytes;
-        const uint32_t kb = sbase + Cfg::kSmemK + s * Cfg::kTileBytes;
+        const uint64_t qa = dQ0 + uint64_t((t * Cfg::kTileBytes) >> 4);
+        const uint64_t kb = dK0 + uint64_t((s * Cfg::kTileBytes) >> 4);
+        const uint32_t dst = tmem + t * 128;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cfg::kChunk + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, make_sdesc_sw128(qa + off, 16, 1024),
-                 make_sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+            mma_ss(dst, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_sfull(t));
         }
-        mma_commit(bar_sfull(t));
+        __syncwarp();
         return true;
+      };
+      auto issue_pv = [&](int t, int j, int s) {
+        const int jlo_t = t ? jlo1 : jlo0;
+        const uint32_t pbase = kSepP ? tmem + Cfg::kColP + t * 64 : tmem + t * 128;
+        const uint32_t dst = tmem + Cfg::kColO + t * D;
+        const uint64_t vb = dV0 + uint64_t((s * Cfg::kTileBytes) >> 4);
+        const uint32_t acc0 = j > jlo_t ? 1u : 0u;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            // P_t: 16 keys of 16-bit values = 8 tensor-memory columns per step
+            mma_ts(dst, pbase + kk * 8, vb + uint64_t((kk * 16 * 128) >> 4), idesc_pv,
+                   kk > 0 ? 1u : acc0);
+          }
+          mma_commit(bar_odone(t));
+        }
+        __syncwarp();
       };
       for (int t = 0; t < 2 && ok; ++t)
         if (in_range(t, JLO)) ok = issue_s(t, JLO);
       for (int j = JLO; j < JHI && ok; ++j) {
         const int idx = j - JLO, s = idx % S, u = idx / S;
         bool v_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (in_range(t, j)) {
+        if constexpr (kSepP) {
+          // S_t(j+1) as soon as the softmax has read S_t(j); then the P V products
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!in_range(t, j + 1)) continue;
+            if (in_range(t, j)) {
+              const int jlo_t = t ? jlo1 : jlo0;
+              ok = wait_all(bar_sfree(t), (j - jlo_t) & 1);
+            }
+            if (ok) ok = issue_s(t, j + 1);
+          }
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!in_range(t, j)) continue;
             if (!v_ready) {
-              ok = mbar_wait(bar_vfull(s), u & 1, wc);
+              ok = wait_all(bar_vfull(s), u & 1);
               v_ready = true;
             }
             const int jlo_t = t ? jlo1 : jlo0;
-            if (ok) ok = mbar_wait(bar_pfull(t), (j - jlo_t) & 1, wc);
+            if (ok) ok = wait_all(bar_pfull(t), (j - jlo_t) & 1);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vb = sbase + Cfg::kSmemV + s * Cfg::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 128 / 16; ++kk) {
-              // P_t: 16 keys of 16-bit values = 8 tensor-memory columns per step
-              mma_ts(tmem + Cfg::kColO + t * D, tmem + t * 128 + kk * 8,
-                     make_sdesc_sw128(vb + kk * 16 * 128, Cfg::kChunk, 1024), idesc_pv,
-                     (j > jlo_t || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(bar_odone(t));
+            issue_pv(t, j, s);
           }
-          if (ok && in_range(t, j + 1)) ok = issue_s(t, j + 1);
+        } else {
+          // P_t aliases S_t: S_t(j+1) follows P_t V_j in the tensor pipe
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (in_range(t, j)) {
+              if (!v_ready) {
+                ok = wait_all(bar_vfull(s), u & 1);
+                v_ready = true;
+              }
+              const int jlo_t = t ? jlo1 : jlo0;
+              if (ok) ok = wait_all(bar_pfull(t), (j - jlo_t) & 1);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, j, s);
+            }
+            if (ok && in_range(t, j + 1)) ok = issue_s(t, j + 1);
+          }
         }
         if (!ok) break;
-        mma_commit(bar_kempty(s));
-        mma_commit(bar_vempty(s));
+        if (elect_one()) {
+          mma_commit(bar_kempty(s));
+          mma_commit(bar_vempty(s));
+        }
+        __syncwarp();
       }
     }
   } else {
@@ -246,6 +351,7 @@ __global__ void __launch_bounds__(320, 1)
     const int row = mblock * 256 + t * 128 + r;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tP = kSepP ? tmem + lane_base + Cfg::kColP + t * 64 : tS;
     const uint32_t tO = tmem + lane_base + Cfg::kColO + t * D;
     int lo_i, hi_i;
     row_key_range(row, p.Nq, p.Nk, p.causal, p.wl, p.wr, lo_i, hi_i);
@@ -266,6 +372,10 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(tS + 64, sr2);
       tmem_ld32(tS + 96, sr3);
       tmem_wait_ld();
+      if constexpr (kSepP) {  // S_t is in registers: the next S_t may be computed
+        tc_fence_before();
+        mbar_arrive(bar_sfree(t));
+      }
       float s[128];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -281,9 +391,18 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < 128; ++c)
           s[c] = (key0 + c >= lo_i && key0 + c <= hi_i) ? s[c] : -INFINITY;
       }
-      float mx = s[0];
+      // row max as a tree of 3-input maxima (no long dependent chain)
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int e = 0; e < 8; ++e) mx8[e] = fmax3(s[e], s[e + 8], s[e + 16]);
+#pragma unroll
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], s[c + e], s[c + 8 + e]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[120 + e]);
+      const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                             fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
       const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sc;
       const float m_new = fmaxf(m_use, m_tile);
       const bool grow = m_new > m_use + 8.0f || (m_use == -INFINITY && m_new != -INFINITY);
@@ -293,30 +412,48 @@ __global__ void __launch_bounds__(320, 1)
         m_use = m_new;
         l *= alpha;
       }
+      // P = exp2(S * scale * log2 e - m), packed to 16 bit; a fixed share of
+      // the column pairs takes the FMA-pipe exp2, the rest the MUFU ex2
       const float base = (m_use == -INFINITY) ? 0.f : m_use;
-      float l0 = 0.f, l1 = 0.f;
-      uint32_t pk0[32], pk1[32];
+      const float2 sc2 = make_float2(sc, sc);
+      const float2 nb2 = make_float2(-base, -base);
+      float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = fast_exp2(fmaf(s[2 * c], sc, -base));
-        const float p1 = fast_exp2(fmaf(s[2 * c + 1], sc, -base));
-        const float p2 = fast_exp2(fmaf(s[64 + 2 * c], sc, -base));
-        const float p3 = fast_exp2(fmaf(s[64 + 2 * c + 1], sc, -base));
-        l0 += p0 + p1;
-        l1 += p2 + p3;
-        pk0[c] = pack2<BF16>(p0, p1);
-        pk1[c] = pack2<BF16>(p2, p3);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int cc = 32 * half + c;  // column pair
+          const float2 x = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), sc2, nb2);
+          float2 pv;
+          if ((cc & 7) < Cfg::kEmuPairsPer8) {
+            pv = exp2_fma_pair<BF16>(x);
+          } else {
+            pv.x = fast_exp2(x.x);
+            pv.y = fast_exp2(x.y);
+          }
+          lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);
+          pk[c] = pack2<BF16>(pv.x, pv.y);
+        }
+        // P_t V_{j-1} must be complete before P_t is rewritten (with P over S
+        // this is implied: S_t(j) itself followed P_t V_{j-1} in the pipe)
+        if (kSepP && half == 0 && jj > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(t), (jj - 1) & 1, wc));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        tmem_st32(tP + 32 * half, pk);
       }
-      l += l0 + l1;
-      tmem_st32(tS + 0, pk0);
-      tmem_st32(tS + 32, pk1);
-      tmem_wait_st();
+      if (!ok) break;
+      const float2 ls2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
+      l += ls2.x + ls2.y;
       if (jj > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_t must hold P_{j-1} V_{j-1} before it is rescaled (S is consumed by
-        // now, which keeps register pressure low here)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(t), (jj - 1) & 1, wc));
-        if (!ok) break;
-        tc_fence_after();
+        if constexpr (!kSepP) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(t), (jj - 1) & 1, wc));
+          if (!ok) break;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t orr[32];
@@ -339,9 +476,8 @@ __global__ void __launch_bounds__(320, 1)
       const float inv_l = has ? 1.f / l : 0.f;
       const float lse = has ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const bool store = row < p.Nq;
-      using elem_t = uint16_t;
-      elem_t* orow = reinterpret_cast<elem_t*>(p.o) + b * p.o_sb + int64_t(row) * p.o_ss +
-                     int64_t(h) * p.o_sh;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + b * p.o_sb + int64_t(row) * p.o_ss +
+                       int64_t(h) * p.o_sh;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t orr[32];

@@ -194,6 +194,18 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
   return desc;
 }
 
+// Constant (non-address) part of a 128-byte-swizzle descriptor; OR-ing in
+// (smem address >> 4) gives the full descriptor.  Shared-memory addresses stay
+// below 2^18, so (address >> 4) fits the 14-bit field and later offsets can be
+// added to the descriptor directly (no carry leaves the field).
+__host__ __device__ constexpr uint64_t sdesc_sw128_const(uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return (uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16) | (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t desc_const, uint32_t saddr) {
+  return desc_const | uint64_t((saddr >> 4) & 0x3FFFu);
+}
+
 // 32 lanes x 32 columns of 32-bit words: thread t of the warp gets lane
 // (warp's lane quarter)*32 + t, columns col..col+31.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -228,6 +240,20 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// One lane of a converged warp (the lowest active lane, so the same lane on
+// every call): it issues the warp's tcgen05 MMAs and commits.  Keeping the
+// warp converged around the MMAs keeps their operands warp-uniform, which
+// issues far faster than MMAs from a lane running alone.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // Named barrier among `nthreads` threads (multiple of 32).
