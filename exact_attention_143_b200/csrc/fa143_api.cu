@@ -96,7 +96,8 @@ int check_common(int B, int Nq, int Nk, int Hq, int Hkv, int d, int dtype, float
   if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   // grid and TMA coordinate limits
-  if (Nq > (1 << 24) || Nk > (1 << 24) || int64_t(B) * Hq > (int64_t(1) << 30))
+  if (Nq > (1 << 24) || Nk > (1 << 24) || int64_t(B) * Hq > (int64_t(1) << 30) ||
+      (Nq + 255) / 256 > 65535 || (Nk + 127) / 128 > 65535)
     return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
@@ -153,9 +154,28 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// 3-D fp32 tensor map over the dQ accumulator [B*Hq, Nq, d] for the bulk
+// reduce-adds: box of 32 columns (128 B, 128-byte swizzle) x rows_per_box rows.
+int make_dq_acc_map(CUtensorMap* map, float* dq_acc, int B, int Nq, int Hq, int d,
+                    int rows_per_box) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(Nq), cuuint64_t(B) * cuuint64_t(Hq)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(Nq) * cuuint64_t(d) * 4};
+  cuuint32_t box[3] = {32, cuuint32_t(rows_per_box), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D, bool BF16>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mdo, const fa::BwdParams& prm, cudaStream_t st) {
+  CUtensorMap mdq;
+  int rc = make_dq_acc_map(&mdq, prm.dq_acc, prm.B, prm.Nq, prm.Hq, D, 128);
+  if (rc) return rc;
   using Cfg = fa::BwdCfg<D>;
   auto kern = fa::fa_bwd_main_kernel<D, BF16>;
   static bool attr_done = false;  // per instantiation and process
@@ -166,7 +186,7 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     attr_done = true;
   }
   dim3 grid(unsigned(prm.B * prm.Hkv), unsigned(prm.n_ntiles));
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mdo, prm);
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -26,14 +26,19 @@
 //                                                    smem as the dQ operand)
 //        dK  += dS^T Q_i       (A = dS^T from tensor memory)
 //        dQ_i = dS K           (A = dS from smem, MN-major)
-//      and the dQ warps add scale * dQ_i into the fp32 accumulator.
+//      and the compute warps add scale * dQ_i into the fp32 accumulator with
+//      TMA bulk reduce-adds staged through shared memory.
 //   3. fa_bwd_dq_convert_kernel: dQ accumulator -> dQ in the input dtype.
 //
-// Roles (320 threads): warps 0-3 compute (thread = key row = tensor-memory
-// lane), warps 4-7 dQ readout (thread = query row), warp 8 MMA issuer,
-// warp 9 TMA producer.  Tensor memory: two 128-column regions R0/R1 swap
-// roles every step (S/P/dQ in one, dP/dS in the other), dK at 256, dV at
-// 256 + d.
+// Roles (448 threads): warps 0-7 compute (thread = key row = tensor-memory
+// lane; warps 0-3 take queries 0-63 of a tile, warps 4-7 queries 64-127),
+// warps 8-11 move dQ out of tensor memory and reduce it into the fp32
+// accumulator, warp 12 issues the MMAs (one elected lane of a converged warp),
+// warp 13 issues TMA loads.
+// Tensor memory: two 128-column regions R0/R1 swap roles every step (S, P, dQ
+// in one; dP, dS in the other), dK at 256, dV at 256 + d.  Per step the MMA
+// order is dV(s), dK(s), S(s+1), dQ(s), dP(s+1); dQ(s) is reduced while the
+// compute warps work on step s+1.
 #pragma once
 
 #include <climits>
@@ -154,7 +159,7 @@ template <int D>
 struct BwdCfg {
   static constexpr int kChunk = 128 * 64 * 2;     // 128 rows x 64 columns, 16-bit, swizzled
   static constexpr int kTileBytes = 128 * D * 2;  // a 128-row tile
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 448;
   static constexpr int kSmemK = 0;
   static constexpr int kSmemV = kSmemK + kTileBytes;
   static constexpr int kSmemQ = kSmemV + kTileBytes;        // 2 stages
@@ -167,6 +172,7 @@ struct BwdCfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = 256 + D;
+  static constexpr int kDqRounds = D / 64;  // 64 dQ columns (2 boxes of 32) per reduce round
 };
 
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
@@ -179,11 +185,12 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
-                       const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmDO,
+                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using Cfg = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -201,6 +208,9 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t bar_ds = smem_u32(&bars[8]);
   const uint32_t bar_dq = smem_u32(&bars[9]);
   const uint32_t bar_dqfree = smem_u32(&bars[10]);
+  const uint32_t bar_staged = smem_u32(&bars[11]);     // a dQ round staged (128 arrivals)
+  const uint32_t bar_roundfree = smem_u32(&bars[12]);  // staged round read by the TMA unit
+  const uint32_t bar_stepfree = smem_u32(&bars[13]);   // whole dQ(s) read: dS buffer free
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kSmemBar + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kSmemBar + 136);
 
@@ -208,6 +218,8 @@ __global__ void __launch_bounds__(320, 1)
   const int lane = threadIdx.x & 31;
 
   // work unit: (batch, kv head) from blockIdx.x, key tile from blockIdx.y
+  // (under a causal mask the first key tiles see the most queries and are
+  // launched first)
   const int bg = blockIdx.x;
   const int g = bg % p.Hkv;
   const int b = bg / p.Hkv;
@@ -235,16 +247,19 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
-    mbar_init(bar_p, 128);
-    mbar_init(bar_ds, 128);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
     mbar_init(bar_dq, 1);
     mbar_init(bar_dqfree, 128);
+    mbar_init(bar_staged, 128);
+    mbar_init(bar_roundfree, 1);
+    mbar_init(bar_stepfree, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
   __syncwarp();
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -256,13 +271,14 @@ __global__ void __launch_bounds__(320, 1)
   auto step_head = [&](int s) { return g * G + s / nm; };
   auto step_mtile = [&](int s) { return mlo + s % nm; };
 
-  if (warp == 9) {
+  if (warp == 13) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && T > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmDQ);
       mbar_arrive_expect_tx(bar_kv, 2 * Cfg::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
         tma_load_4d(sbase + Cfg::kSmemK + c * Cfg::kChunk, &tmK, bar_kv, c * 64, key0, g, b);
@@ -284,7 +300,7 @@ __global__ void __launch_bounds__(320, 1)
         bulk_load_1d(sbase + Cfg::kSmemDv + st * 512, p.Dvec + rowoff, 512, bar_qfull(st));
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop and waits; one elected lane issues each
     // batch of MMAs and its commits.
@@ -306,69 +322,158 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
       const uint64_t dDO_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
       const uint64_t dDO_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
-      bool ok = wait_all(bar_kv, 0);
-      for (int s = 0; s < T && ok; ++s) {
-        const int st = s & 1, u = s >> 1;
-        const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
-        const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
-        if (!(ok = wait_all(bar_qfull(st), u & 1))) break;
-        tc_fence_after();
-        // S^T = K Q^T (M = keys, N = queries, K-dim = d)
+      // S^T(s) = K Q_s^T into region r (M = keys, N = queries, K-dim = d)
+      auto issue_s = [&](int s, uint32_t r) {
+        const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(Ra, dK_k + o, dQ_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
+            mma_ss(r, dK_k + o, dQ_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_s);
         }
         __syncwarp();
-        // dP^T = V dO^T, into the region the previous dQ used
-        if (s > 0 && !(ok = wait_all(bar_dqfree, (s - 1) & 1))) break;
-        tc_fence_after();
+      };
+      // dP^T(s) = V dO_s^T into region r
+      auto issue_dp = [&](int s, uint32_t r) {
+        const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(Rb, dV_k + o, dDO_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
+            mma_ss(r, dV_k + o, dDO_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_dp);
         }
         __syncwarp();
+      };
+      // P^T and dS^T sit in columns [0, 32) (queries 0-63) and [64, 96)
+      // (queries 64-127) of their region: 16 queries per K step = 8 columns
+      auto acol = [](int kk) { return uint32_t(kk < 4 ? kk * 8 : 64 + (kk - 4) * 8); };
+      bool ok = wait_all(bar_kv, 0);
+      if (ok) ok = wait_all(bar_qfull(0), 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, tmem);
+        issue_dp(0, tmem + 128);
+      }
+      for (int s = 0; s < T && ok; ++s) {
+        const int st = s & 1;
+        const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
+        const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
+        const uint32_t acc0 = s > 0 ? 1u : 0u;
         // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major)
         if (!(ok = wait_all(bar_p, s & 1))) break;
         tc_fence_after();
-        const uint32_t acc0 = s > 0 ? 1u : 0u;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Cfg::kColDV, Ra + kk * 8,
+            mma_ts(tmem + Cfg::kColDV, Ra + acol(kk),
                    dDO_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
         }
         __syncwarp();
-        // dK += dS^T Q ; dQ = dS K
+        // dK += dS^T Q (A = dS^T from tensor memory, B = Q MN-major)
         if (!(ok = wait_all(bar_ds, s & 1))) break;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Cfg::kColDK, Rb + kk * 8,
+            mma_ts(tmem + Cfg::kColDK, Rb + acol(kk),
                    dQ_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
+          mma_commit(bar_qempty(st));  // Q_s, dO_s, LSE_s, D_s are no longer read
+        }
+        __syncwarp();
+        // S^T(s+1) into Rb (its dS^T has just been consumed by dK)
+        if (s + 1 < T) {
+          if (!(ok = wait_all(bar_qfull((s + 1) & 1), ((s + 1) >> 1) & 1))) break;
+          tc_fence_after();
+          issue_s(s + 1, Rb);
+        }
+        // dQ(s) = dS K into Ra (A = dS from smem, MN-major; B = K MN-major)
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(Ra, dDS_mn + uint64_t((kk * 2048) >> 4), dK_mn + uint64_t((kk * 2048) >> 4),
                    idesc_dq, kk > 0 ? 1u : 0u);
           mma_commit(bar_dq);
-          mma_commit(bar_qempty(st));
+        }
+        __syncwarp();
+        // dP^T(s+1) into Ra once dQ(s) has been read out of it
+        if (s + 1 < T) {
+          if (!(ok = wait_all(bar_dqfree, s & 1))) break;
+          tc_fence_after();
+          issue_dp(s + 1, Ra);
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ reduction (warps 8-11)
+    // dQ(s) leaves tensor memory (thread = query row r) and scale * dQ(s) is
+    // added into the fp32 accumulator by the TMA unit: per round, 64 columns
+    // of all 128 rows are staged, 128-byte swizzled, in the dS buffer (free
+    // from the end of the dQ(s) MMA until the compute warps write dS(s+1))
+    // and reduced with two bulk tensor reduce-adds of 32 columns each.
+    const int r = threadIdx.x - 256;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+    };
+    uint8_t* stage = smem + Cfg::kSmemDS;
+    constexpr int kR = Cfg::kDqRounds;
+    bool ok = true;
+    for (int s = 0; s < T && ok; ++s) {
+      if (!(ok = wait_all(bar_dq, s & 1))) break;
+      tc_fence_after();
+      const uint32_t R = tmem + lane_base + (s & 1) * 128;
+      const int h = step_head(s), m = step_mtile(s);
+      uint32_t v[64];
+      for (int rd = 0; rd < kR && ok; ++rd) {
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32)
+          tmem_ld32(R + rd * 64 + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+        tmem_wait_ld();
+        if (rd == kR - 1) {  // dQ(s) is out of tensor memory: the region may be reused
+          tc_fence_before();
+          mbar_arrive(bar_dqfree);
+        }
+        // the previous round's staging must have been read by the TMA unit
+        const int prev = s * kR + rd - 1;
+        if (prev >= 0 && !(ok = wait_all(bar_roundfree, prev & 1))) break;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint8_t* chunk = stage + c * (128 * 128) + r * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float* x = reinterpret_cast<const float*>(&v[c * 32 + u * 4]);
+            *reinterpret_cast<float4*>(chunk + ((u ^ (r & 7)) * 16)) =
+                make_float4(x[0] * p.scale, x[1] * p.scale, x[2] * p.scale, x[3] * p.scale);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_staged);
+        if (r == 0 && mbar_wait(bar_staged, uint32_t(s * kR + rd) & 1u, wc)) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tma_reduce_add_3d(&tmDQ, smem_u32(stage) + c * (128 * 128), rd * 64 + c * 32,
+                              m * 128, b * p.Hq + h);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(bar_roundfree);
+          if (rd == kR - 1) mbar_arrive(bar_stepfree);
         }
         __syncwarp();
       }
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ compute: P^T, dS^T
-    const int j = threadIdx.x;  // key row within the tile == tensor-memory lane
+    if (r == 0) bulk_wait0();  // reduce-adds complete before the CTA exits
+  } else {
+    // ------------------------------------------------------------ compute (warps 0-7)
+    const int half = warp >> 2;                 // query half of every tile
+    const int j = (warp & 3) * 32 + lane;       // key row == tensor-memory lane
     const int key = key0 + j;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t colS = half * 64;            // S^T / dP^T columns of this half
+    const uint32_t colP = half * 64;            // packed P^T / dS^T: [colP, colP + 32)
     // queries that see this key: [qlo, qhi]
     int qlo = right >= 0 ? key - off - right : INT_MIN;
     int qhi = p.wl >= 0 ? key - off + p.wl : INT_MAX;
@@ -377,23 +482,25 @@ __global__ void __launch_bounds__(320, 1)
       qhi = INT_MIN;
     }
     const float sc = p.scale_log2;
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+    };
     bool ok = true;
     for (int s = 0; s < T; ++s) {
       const int st = s & 1;
       const uint32_t Ra = tmem + lane_base + (s & 1) * 128;
       const uint32_t Rb = tmem + lane_base + ((s + 1) & 1) * 128;
-      const float* lse2 = reinterpret_cast<const float*>(smem + Cfg::kSmemLSE + st * 512);
-      const float* Dv = reinterpret_cast<const float*>(smem + Cfg::kSmemDv + st * 512);
-      const int q0 = step_mtile(s) * 128;
-      const bool need_mask = __any_sync(0xffffffffu, qlo > q0 || qhi < q0 + 127);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s, s & 1, wc));
-      if (!ok) break;
+      const float* lse2 = reinterpret_cast<const float*>(smem + Cfg::kSmemLSE + st * 512) + half * 64;
+      const float* Dv = reinterpret_cast<const float*>(smem + Cfg::kSmemDv + st * 512) + half * 64;
+      const int q0 = step_mtile(s) * 128 + half * 64;
+      const bool need_mask = __any_sync(0xffffffffu, qlo > q0 || qhi < q0 + 63);
+      if (!(ok = wait_all(bar_s, s & 1))) break;
       tc_fence_after();
       // P^T = exp2(S^T * scale * log2 e - LSE2), 32 queries at a time
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t sr[32];
-        tmem_ld32(Ra + c0, sr);
+        tmem_ld32(Ra + colS + c0, sr);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -414,35 +521,23 @@ __global__ void __launch_bounds__(320, 1)
           pk[c / 2] = pack2<BF16>(pv[0], pv[1]);
           pk[c / 2 + 1] = pack2<BF16>(pv[2], pv[3]);
         }
-        // P^T packed: 32 queries -> 16 columns, written over columns already read
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(Ra + c0 / 2),
-            "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
-            "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
-            "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-            : "memory");
+        // packed P^T written over S^T columns this thread has already read
+        tmem_st16(Ra + colP + c0 / 2, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
-      // dS^T = P^T * (dP^T - D); the smem copy waits until the previous dQ MMA is done
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, s & 1, wc));
-      if (ok && s > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (s - 1) & 1, wc));
-      if (!ok) break;
+      // dS^T = P^T * (dP^T - D), to tensor memory and to smem (dQ operand);
+      // the smem buffer is free once dQ(s-1) has been staged and read
+      if (!(ok = wait_all(bar_dp, s & 1))) break;
+      if (s > 0 && !(ok = wait_all(bar_stepfree, (s - 1) & 1))) break;
       tc_fence_after();
-      uint8_t* dsrow = smem + Cfg::kSmemDS + j * 128;
+      uint8_t* dsrow = smem + Cfg::kSmemDS + half * Cfg::kChunk + j * 128;
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t dpr[32], pr[16];
-        tmem_ld32(Rb + c0, dpr);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(pr[0]), "=r"(pr[1]), "=r"(pr[2]), "=r"(pr[3]), "=r"(pr[4]), "=r"(pr[5]),
-              "=r"(pr[6]), "=r"(pr[7]), "=r"(pr[8]), "=r"(pr[9]), "=r"(pr[10]), "=r"(pr[11]),
-              "=r"(pr[12]), "=r"(pr[13]), "=r"(pr[14]), "=r"(pr[15])
-            : "r"(Ra + c0 / 2));
+        tmem_ld32(Rb + colS + c0, dpr);
+        tmem_ld16(Ra + colP + c0 / 2, pr);
         tmem_wait_ld();
         uint32_t dk[16];
 #pragma unroll
@@ -469,22 +564,15 @@ __global__ void __launch_bounds__(320, 1)
           dk[c / 2] = pack2<BF16>(ds0, ds1);
           dk[c / 2 + 1] = pack2<BF16>(ds2, ds3);
         }
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(Rb + c0 / 2),
-            "r"(dk[0]), "r"(dk[1]), "r"(dk[2]), "r"(dk[3]), "r"(dk[4]), "r"(dk[5]), "r"(dk[6]),
-            "r"(dk[7]), "r"(dk[8]), "r"(dk[9]), "r"(dk[10]), "r"(dk[11]), "r"(dk[12]),
-            "r"(dk[13]), "r"(dk[14]), "r"(dk[15])
-            : "memory");
+        tmem_st16(Rb + colP + c0 / 2, dk);
         // smem copy in the MN-major 128-byte-swizzled layout of the dQ A operand:
-        // chunk (c0 / 64) holds queries [64 chunk, +64) of every key row; the
-        // 16-byte unit u of row j sits at unit u ^ (j % 8).
-        uint8_t* chunk = dsrow + (c0 >> 6) * Cfg::kChunk;
-        const int u0 = (c0 & 63) >> 3;  // first 16-byte unit of these 32 queries
+        // chunk `half` holds queries [64 half, 64 half + 64) of every key row;
+        // the 16-byte unit u of row j sits at unit u ^ (j % 8).
+        const int u0 = c0 >> 3;
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
           const int u = (u0 + uu) ^ (j & 7);
-          *reinterpret_cast<uint4*>(chunk + u * 16) =
+          *reinterpret_cast<uint4*>(dsrow + u * 16) =
               make_uint4(dk[4 * uu], dk[4 * uu + 1], dk[4 * uu + 2], dk[4 * uu + 3]);
         }
       }
@@ -493,22 +581,23 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(bar_ds);
     }
-    // epilogue: dK = scale * (dS^T Q summed), dV = (P^T dO summed), in the input dtype
-    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (T - 1) & 1, wc));
+    if (ok && T > 0) ok = wait_all(bar_dq, (T - 1) & 1);  // every MMA of this CTA is done
+    // epilogue: dK = scale * (sum of dS^T Q), dV = sum of P^T dO, in the input
+    // dtype; this thread writes half of the columns of key row j
     if (ok) {
       tc_fence_after();
       const bool store = key < p.Nk;
       uint16_t* dkrow = static_cast<uint16_t*>(p.dk) + b * p.dk_sb + int64_t(key) * p.dk_ss +
-                        int64_t(g) * p.dk_sh;
+                        int64_t(g) * p.dk_sh + half * (D / 2);
       uint16_t* dvrow = static_cast<uint16_t*>(p.dv) + b * p.dv_sb + int64_t(key) * p.dv_ss +
-                        int64_t(g) * p.dv_sh;
+                        int64_t(g) * p.dv_sh + half * (D / 2);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? Cfg::kColDK : Cfg::kColDV;
+        const uint32_t col = (which == 0 ? Cfg::kColDK : Cfg::kColDV) + half * (D / 2);
         const float mul = which == 0 ? p.scale : 1.f;
         uint16_t* dst_row = which == 0 ? dkrow : dvrow;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
           uint32_t r[32];
           if (T > 0) {
             tmem_ld32(tmem + lane_base + col + c0, r);
@@ -531,37 +620,12 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  } else {
-    // ------------------------------------------------------------ dQ readout (warps 4-7)
-    const int r = threadIdx.x - 128;  // query row within the tile == tensor-memory lane
-    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    for (int s = 0; s < T; ++s) {
-      const uint32_t Ra = tmem + lane_base + (s & 1) * 128;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, s & 1, wc))) break;
-      tc_fence_after();
-      uint32_t v[D];
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(Ra + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_dqfree);
-      const int h = step_head(s), row = step_mtile(s) * 128 + r;
-      if (row < p.Nq) {
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((int64_t(b) * p.Hq + h) * p.Nq + row) * D);
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c)
-          atomicAdd(dst + c, make_float4(__uint_as_float(v[4 * c]) * p.scale,
-                                         __uint_as_float(v[4 * c + 1]) * p.scale,
-                                         __uint_as_float(v[4 * c + 2]) * p.scale,
-                                         __uint_as_float(v[4 * c + 3]) * p.scale));
-      }
-    }
   }
 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }
