@@ -178,12 +178,25 @@ def dist_setup(args):
 
 
 def dist_max(x, world):
+    """Max of x over all ranks (CPU tensor under gloo, CUDA tensor under nccl)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([float(x)], device="cuda")
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_workload(w: Workload, rank: int) -> Workload:
+    """Each rank runs an independent replica of the workload (its own seed)."""
+    return Workload(**{**w.__dict__, "seed": w.seed + rank})
+
+
+def aggregate_tflops(world, flops_per_step, steps, max_total_ms):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return world * flops_per_step * steps / (max_total_ms / 1e3) / 1e12
 
 
 def dist_barrier(world):
@@ -250,7 +263,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
 
     # inputs (each rank an independent replica: seed + rank), resident in HBM
-    wr = Workload(**{**w.__dict__, "seed": w.seed + rank})
+    wr = replica_workload(w, rank)
     q, k, v, do = make_workload_inputs(wr, with_dout=True)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o = torch.empty_like(qd)
@@ -295,7 +308,7 @@ def run_ours(args):
     total_ms_max = dist_max(total_ms, world)
     f_fwd = fwd_flops(w)
     f_step = 3.5 * f_fwd
-    value = world * f_step * K / (total_ms_max / 1e3) / 1e12
+    value = aggregate_tflops(world, f_step, K, total_ms_max)
     bwd_main_avg = sum(main_ms) / K
     achieved = 2.5 * f_fwd / (bwd_main_avg / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
@@ -324,7 +337,7 @@ def run_ours(args):
         e_ms = dist_max(sum(ems), world)
         h2d = sum(t.numel() * t.element_size() for t in (q, k, v, do))
         d2h = sum(t.numel() * t.element_size() for t in (dq, dk, dv))
-        e2e = {"value": world * f_step * Ke / (e_ms / 1e3) / 1e12, "unit": "TFLOPS",
+        e2e = {"value": aggregate_tflops(world, f_step, Ke, e_ms), "unit": "TFLOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
 
     # per-workload forward table (rank 0, N = 1 only): each pages' config alone
