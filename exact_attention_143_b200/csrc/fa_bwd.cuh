@@ -30,11 +30,13 @@
 //      TMA bulk reduce-adds staged through shared memory.
 //   3. fa_bwd_dq_convert_kernel: dQ accumulator -> dQ in the input dtype.
 //
-// Roles (448 threads): warps 0-7 compute (thread = key row = tensor-memory
+// Roles (480 threads): warps 0-7 compute (thread = key row = tensor-memory
 // lane; warps 0-3 take queries 0-63 of a tile, warps 4-7 queries 64-127),
-// warps 8-11 move dQ out of tensor memory and reduce it into the fp32
-// accumulator, warp 12 issues the MMAs (one elected lane of a converged warp),
-// warp 13 issues TMA loads.
+// warps 8-11 move dQ out of tensor memory into a staging buffer, warp 14
+// reduces the staged rows into the fp32 accumulator (TMA bulk reduce-add),
+// warp 12 issues the MMAs (one elected lane of a converged warp), warp 13
+// issues TMA loads.  dO has one buffer, refilled as soon as dV has read it;
+// that frees the staging buffer so the compute warps never wait for dQ.
 // Tensor memory: two 128-column regions R0/R1 swap roles every step (S, P, dQ
 // in one; dP, dS in the other), dK at 256, dV at 256 + d.  Per step the MMA
 // order is dV(s), dK(s), S(s+1), dQ(s), dP(s+1); dQ(s) is reduced while the
@@ -46,6 +48,7 @@
 #include <cuda_fp16.h>
 
 #include "fa_ptx.cuh"
+#include "fa_fwd.cuh"  // exp2_fma_pair
 
 namespace fa {
 
@@ -159,13 +162,14 @@ template <int D>
 struct BwdCfg {
   static constexpr int kChunk = 128 * 64 * 2;     // 128 rows x 64 columns, 16-bit, swizzled
   static constexpr int kTileBytes = 128 * D * 2;  // a 128-row tile
-  static constexpr int kThreads = 448;
+  static constexpr int kThreads = 480;
   static constexpr int kSmemK = 0;
   static constexpr int kSmemV = kSmemK + kTileBytes;
   static constexpr int kSmemQ = kSmemV + kTileBytes;        // 2 stages
-  static constexpr int kSmemDO = kSmemQ + 2 * kTileBytes;   // 2 stages
-  static constexpr int kSmemDS = kSmemDO + 2 * kTileBytes;  // 128 keys x 128 queries, 16-bit
-  static constexpr int kSmemLSE = kSmemDS + 2 * kChunk;     // 2 stages x 128 fp32
+  static constexpr int kSmemDO = kSmemQ + 2 * kTileBytes;   // 1 stage
+  static constexpr int kSmemDS = kSmemDO + kTileBytes;      // 128 keys x 128 queries, 16-bit
+  static constexpr int kSmemSTG = kSmemDS + 2 * kChunk;     // dQ staging: 128 rows x 64 fp32
+  static constexpr int kSmemLSE = kSmemSTG + 32768;         // 2 stages x 128 fp32
   static constexpr int kSmemDv = kSmemLSE + 2 * 512;        // 2 stages x 128 fp32
   static constexpr int kSmemBar = kSmemDv + 2 * 512;
   static constexpr int kSmemBytes = kSmemBar + 256;
@@ -173,6 +177,8 @@ struct BwdCfg {
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = 256 + D;
   static constexpr int kDqRounds = D / 64;  // 64 dQ columns (2 boxes of 32) per reduce round
+  // of every 8 query pairs of a row, how many take the FMA-pipe exp2
+  static constexpr int kEmuPairsPer8 = 2;
 };
 
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
@@ -185,7 +191,7 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(480, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
@@ -200,19 +206,20 @@ __global__ void __launch_bounds__(448, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kSmemBar);
   const uint32_t bar_kv = smem_u32(&bars[0]);
-  auto bar_qfull = [&](int st) { return smem_u32(&bars[1 + st]); };
+  auto bar_qfull = [&](int st) { return smem_u32(&bars[1 + st]); };   // Q, LSE2, D of a step
   auto bar_qempty = [&](int st) { return smem_u32(&bars[3 + st]); };
-  const uint32_t bar_s = smem_u32(&bars[5]);
-  const uint32_t bar_dp = smem_u32(&bars[6]);
-  const uint32_t bar_p = smem_u32(&bars[7]);
-  const uint32_t bar_ds = smem_u32(&bars[8]);
-  const uint32_t bar_dq = smem_u32(&bars[9]);
-  const uint32_t bar_dqfree = smem_u32(&bars[10]);
-  const uint32_t bar_staged = smem_u32(&bars[11]);     // a dQ round staged (128 arrivals)
-  const uint32_t bar_roundfree = smem_u32(&bars[12]);  // staged round read by the TMA unit
-  const uint32_t bar_stepfree = smem_u32(&bars[13]);   // whole dQ(s) read: dS buffer free
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kSmemBar + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kSmemBar + 136);
+  const uint32_t bar_dofull = smem_u32(&bars[5]);     // dO of a step (one buffer)
+  const uint32_t bar_doempty = smem_u32(&bars[6]);
+  const uint32_t bar_s = smem_u32(&bars[7]);
+  const uint32_t bar_dp = smem_u32(&bars[8]);
+  const uint32_t bar_p = smem_u32(&bars[9]);
+  const uint32_t bar_ds = smem_u32(&bars[10]);
+  const uint32_t bar_dq = smem_u32(&bars[11]);
+  const uint32_t bar_dqfree = smem_u32(&bars[12]);
+  const uint32_t bar_staged = smem_u32(&bars[13]);     // a dQ round staged (128 arrivals)
+  const uint32_t bar_roundfree = smem_u32(&bars[14]);  // staged round read by the TMA unit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kSmemBar + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kSmemBar + 200);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -245,6 +252,8 @@ __global__ void __launch_bounds__(448, 1)
       mbar_init(bar_qfull(st), 1);
       mbar_init(bar_qempty(st), 1);
     }
+    mbar_init(bar_dofull, 1);
+    mbar_init(bar_doempty, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
     mbar_init(bar_p, 256);
@@ -253,7 +262,6 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_dqfree, 128);
     mbar_init(bar_staged, 128);
     mbar_init(bar_roundfree, 1);
-    mbar_init(bar_stepfree, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -270,6 +278,9 @@ __global__ void __launch_bounds__(448, 1)
 
   auto step_head = [&](int s) { return g * G + s / nm; };
   auto step_mtile = [&](int s) { return mlo + s % nm; };
+  auto wait_all = [&](uint32_t bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+  };
 
   if (warp == 13) {
     // ------------------------------------------------------------ TMA producer
@@ -278,7 +289,6 @@ __global__ void __launch_bounds__(448, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
-      tma_prefetch_desc(&tmDQ);
       mbar_arrive_expect_tx(bar_kv, 2 * Cfg::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
         tma_load_4d(sbase + Cfg::kSmemK + c * Cfg::kChunk, &tmK, bar_kv, c * 64, key0, g, b);
@@ -286,19 +296,49 @@ __global__ void __launch_bounds__(448, 1)
       }
       for (int s = 0; s < T; ++s) {
         const int st = s & 1, u = s >> 1;
-        if (u > 0 && !mbar_wait(bar_qempty(st), (u - 1) & 1, wc)) break;
         const int h = step_head(s), m = step_mtile(s);
-        mbar_arrive_expect_tx(bar_qfull(st), 2 * Cfg::kTileBytes + 1024);
-        for (int c = 0; c < D / 64; ++c) {
+        // Q, LSE2 and D: two stages
+        if (u > 0 && !mbar_wait(bar_qempty(st), (u - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(bar_qfull(st), Cfg::kTileBytes + 1024);
+        for (int c = 0; c < D / 64; ++c)
           tma_load_4d(sbase + Cfg::kSmemQ + st * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ,
                       bar_qfull(st), c * 64, m * 128, h, b);
-          tma_load_4d(sbase + Cfg::kSmemDO + st * Cfg::kTileBytes + c * Cfg::kChunk, &tmDO,
-                      bar_qfull(st), c * 64, m * 128, h, b);
-        }
         const int64_t rowoff = (int64_t(b) * p.Hq + h) * p.Nq_pad + int64_t(m) * 128;
         bulk_load_1d(sbase + Cfg::kSmemLSE + st * 512, p.lse2 + rowoff, 512, bar_qfull(st));
         bulk_load_1d(sbase + Cfg::kSmemDv + st * 512, p.Dvec + rowoff, 512, bar_qfull(st));
+        // dO: one buffer, refilled once dV(s-1) has read it
+        if (s > 0 && !mbar_wait(bar_doempty, (s - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(bar_dofull, Cfg::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sbase + Cfg::kSmemDO + c * Cfg::kChunk, &tmDO, bar_dofull, c * 64, m * 128,
+                      h, b);
       }
+    }
+  } else if (warp == 14) {
+    // ------------------------------------------------------------ dQ reduce issuer
+    // Once a round of dQ rows is staged, one elected lane reduces it into the
+    // fp32 accumulator (two bulk tensor reduce-adds of 32 columns x 128 rows)
+    // and reports when the TMA unit has read the staging buffer.
+    if (T > 0) {
+      bool ok = true;
+      for (int s = 0; s < T && ok; ++s) {
+        const int h = step_head(s), m = step_mtile(s);
+        for (int rd = 0; rd < Cfg::kDqRounds && ok; ++rd) {
+          if (!(ok = wait_all(bar_staged, uint32_t(s * Cfg::kDqRounds + rd) & 1u))) break;
+          if (elect_one()) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_reduce_add_3d(&tmDQ, sbase + Cfg::kSmemSTG + c * (128 * 128), rd * 64 + c * 32,
+                                m * 128, b * p.Hq + h);
+            bulk_commit();
+            bulk_wait_read0();
+            mbar_arrive(bar_roundfree);
+          }
+          __syncwarp();
+        }
+      }
+      if (elect_one()) bulk_wait0();  // reduce-adds complete before the CTA exits
+      __syncwarp();
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
@@ -308,9 +348,6 @@ __global__ void __launch_bounds__(448, 1)
       const uint32_t idesc_ss = make_idesc_f16(BF16, 128, 128, false, false);   // S^T, dP^T
       const uint32_t idesc_acc = make_idesc_f16(BF16, 128, D, false, true);    // dV, dK
       const uint32_t idesc_dq = make_idesc_f16(BF16, 128, D, true, true);      // dQ
-      auto wait_all = [&](uint32_t bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
-      };
       // descriptors are built once; an MMA only adds a compile-time offset
       constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
       constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // MN-major tiles
@@ -320,8 +357,8 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t dDS_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDS);
       const uint64_t dQ_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
       const uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
-      const uint64_t dDO_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
-      const uint64_t dDO_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
+      const uint64_t dDO_k = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
+      const uint64_t dDO_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
       // S^T(s) = K Q_s^T into region r (M = keys, N = queries, K-dim = d)
       auto issue_s = [&](int s, uint32_t r) {
         const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
@@ -336,13 +373,12 @@ __global__ void __launch_bounds__(448, 1)
         __syncwarp();
       };
       // dP^T(s) = V dO_s^T into region r
-      auto issue_dp = [&](int s, uint32_t r) {
-        const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
+      auto issue_dp = [&](uint32_t r) {
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(r, dV_k + o, dDO_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
+            mma_ss(r, dV_k + o, dDO_k + o, idesc_ss, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_dp);
         }
@@ -356,21 +392,26 @@ __global__ void __launch_bounds__(448, 1)
       if (ok) {
         tc_fence_after();
         issue_s(0, tmem);
-        issue_dp(0, tmem + 128);
+        ok = wait_all(bar_dofull, 0);
+        if (ok) {
+          tc_fence_after();
+          issue_dp(tmem + 128);
+        }
       }
       for (int s = 0; s < T && ok; ++s) {
         const int st = s & 1;
         const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
         const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
         const uint32_t acc0 = s > 0 ? 1u : 0u;
-        // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major)
+        // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major); dO is then free
         if (!(ok = wait_all(bar_p, s & 1))) break;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Cfg::kColDV, Ra + acol(kk),
-                   dDO_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
+            mma_ts(tmem + Cfg::kColDV, Ra + acol(kk), dDO_mn + uint64_t((kk * 2048) >> 4),
+                   idesc_acc, kk > 0 ? 1u : acc0);
+          mma_commit(bar_doempty);
         }
         __syncwarp();
         // dK += dS^T Q (A = dS^T from tensor memory, B = Q MN-major)
@@ -381,7 +422,7 @@ __global__ void __launch_bounds__(448, 1)
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + Cfg::kColDK, Rb + acol(kk),
                    dQ_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
-          mma_commit(bar_qempty(st));  // Q_s, dO_s, LSE_s, D_s are no longer read
+          mma_commit(bar_qempty(st));  // Q_s, LSE_s, D_s are no longer read
         }
         __syncwarp();
         // S^T(s+1) into Rb (its dS^T has just been consumed by dK)
@@ -399,39 +440,34 @@ __global__ void __launch_bounds__(448, 1)
           mma_commit(bar_dq);
         }
         __syncwarp();
-        // dP^T(s+1) into Ra once dQ(s) has been read out of it
+        // dP^T(s+1) into Ra once dQ(s) has been read out of it and dO(s+1) is in
         if (s + 1 < T) {
           if (!(ok = wait_all(bar_dqfree, s & 1))) break;
+          if (!(ok = wait_all(bar_dofull, (s + 1) & 1))) break;
           tc_fence_after();
-          issue_dp(s + 1, Ra);
+          issue_dp(Ra);
         }
       }
     }
   } else if (warp >= 8) {
-    // ------------------------------------------------------------ dQ reduction (warps 8-11)
-    // dQ(s) leaves tensor memory (thread = query row r) and scale * dQ(s) is
-    // added into the fp32 accumulator by the TMA unit: per round, 64 columns
-    // of all 128 rows are staged, 128-byte swizzled, in the dS buffer (free
-    // from the end of the dQ(s) MMA until the compute warps write dS(s+1))
-    // and reduced with two bulk tensor reduce-adds of 32 columns each.
+    // ------------------------------------------------------------ dQ readout (warps 8-11)
+    // dQ(s) leaves tensor memory (thread = query row r) 64 columns at a time;
+    // scale * dQ is staged, 128-byte swizzled, in the staging buffer for the
+    // reduce issuer.  The tensor-memory region is released right after the
+    // last load, before the staging of the last round.
     const int r = threadIdx.x - 256;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    auto wait_all = [&](uint32_t bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
-    };
-    uint8_t* stage = smem + Cfg::kSmemDS;
+    uint8_t* stage = smem + Cfg::kSmemSTG;
     constexpr int kR = Cfg::kDqRounds;
     bool ok = true;
     for (int s = 0; s < T && ok; ++s) {
       if (!(ok = wait_all(bar_dq, s & 1))) break;
       tc_fence_after();
       const uint32_t R = tmem + lane_base + (s & 1) * 128;
-      const int h = step_head(s), m = step_mtile(s);
-      uint32_t v[64];
       for (int rd = 0; rd < kR && ok; ++rd) {
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32)
-          tmem_ld32(R + rd * 64 + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+        uint32_t v[64];
+        tmem_ld32(R + rd * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(R + rd * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
         if (rd == kR - 1) {  // dQ(s) is out of tensor memory: the region may be reused
           tc_fence_before();
@@ -452,20 +488,8 @@ __global__ void __launch_bounds__(448, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(bar_staged);
-        if (r == 0 && mbar_wait(bar_staged, uint32_t(s * kR + rd) & 1u, wc)) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            tma_reduce_add_3d(&tmDQ, smem_u32(stage) + c * (128 * 128), rd * 64 + c * 32,
-                              m * 128, b * p.Hq + h);
-          bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(bar_roundfree);
-          if (rd == kR - 1) mbar_arrive(bar_stepfree);
-        }
-        __syncwarp();
       }
     }
-    if (r == 0) bulk_wait0();  // reduce-adds complete before the CTA exits
   } else {
     // ------------------------------------------------------------ compute (warps 0-7)
     const int half = warp >> 2;                 // query half of every tile
@@ -481,10 +505,7 @@ __global__ void __launch_bounds__(448, 1)
       qlo = INT_MAX;
       qhi = INT_MIN;
     }
-    const float sc = p.scale_log2;
-    auto wait_all = [&](uint32_t bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
-    };
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int s = 0; s < T; ++s) {
       const int st = s & 1;
@@ -496,7 +517,8 @@ __global__ void __launch_bounds__(448, 1)
       const bool need_mask = __any_sync(0xffffffffu, qlo > q0 || qhi < q0 + 63);
       if (!(ok = wait_all(bar_s, s & 1))) break;
       tc_fence_after();
-      // P^T = exp2(S^T * scale * log2 e - LSE2), 32 queries at a time
+      // P^T = exp2(S^T * scale * log2 e - LSE2), 32 queries at a time; a share
+      // of the query pairs takes the FMA-pipe exp2
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t sr[32];
@@ -506,11 +528,23 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
-          float pv[4];
-          pv[0] = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, -l4.x));
-          pv[1] = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, -l4.y));
-          pv[2] = fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sc, -l4.z));
-          pv[3] = fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sc, -l4.w));
+          const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                        sc2, make_float2(-l4.x, -l4.y));
+          const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])),
+                                        sc2, make_float2(-l4.z, -l4.w));
+          const int pair = (c0 + c) / 2;  // query pair index within this half
+          float2 p01, p23;
+          if ((pair & 7) < Cfg::kEmuPairsPer8) {
+            p01 = exp2_fma_pair<BF16>(x01);
+          } else {
+            p01 = make_float2(fast_exp2(x01.x), fast_exp2(x01.y));
+          }
+          if (((pair + 1) & 7) < Cfg::kEmuPairsPer8) {
+            p23 = exp2_fma_pair<BF16>(x23);
+          } else {
+            p23 = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
+          }
+          float pv[4] = {p01.x, p01.y, p23.x, p23.y};
           if (need_mask) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -528,9 +562,9 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_before();
       mbar_arrive(bar_p);
       // dS^T = P^T * (dP^T - D), to tensor memory and to smem (dQ operand);
-      // the smem buffer is free once dQ(s-1) has been staged and read
+      // the dQ(s-1) MMA, the last reader of the smem buffer, completed before
+      // dP^T(s) was issued
       if (!(ok = wait_all(bar_dp, s & 1))) break;
-      if (s > 0 && !(ok = wait_all(bar_stepfree, (s - 1) & 1))) break;
       tc_fence_after();
       uint8_t* dsrow = smem + Cfg::kSmemDS + half * Cfg::kChunk + j * 128;
 #pragma unroll
@@ -557,12 +591,16 @@ __global__ void __launch_bounds__(448, 1)
             pf[2] = bb.x;
             pf[3] = bb.y;
           }
-          const float ds0 = pf[0] * (__uint_as_float(dpr[c]) - d4.x);
-          const float ds1 = pf[1] * (__uint_as_float(dpr[c + 1]) - d4.y);
-          const float ds2 = pf[2] * (__uint_as_float(dpr[c + 2]) - d4.z);
-          const float ds3 = pf[3] * (__uint_as_float(dpr[c + 3]) - d4.w);
-          dk[c / 2] = pack2<BF16>(ds0, ds1);
-          dk[c / 2 + 1] = pack2<BF16>(ds2, ds3);
+          const float2 d01 = __fmul2_rn(make_float2(pf[0], pf[1]),
+                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c]),
+                                                               __uint_as_float(dpr[c + 1])),
+                                                   make_float2(-d4.x, -d4.y)));
+          const float2 d23 = __fmul2_rn(make_float2(pf[2], pf[3]),
+                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c + 2]),
+                                                               __uint_as_float(dpr[c + 3])),
+                                                   make_float2(-d4.z, -d4.w)));
+          dk[c / 2] = pack2<BF16>(d01.x, d01.y);
+          dk[c / 2 + 1] = pack2<BF16>(d23.x, d23.y);
         }
         tmem_st16(Rb + colP + c0 / 2, dk);
         // smem copy in the MN-major 128-byte-swizzled layout of the dQ A operand:
