@@ -8,12 +8,13 @@
 // with correct normalisation; matmul -> softmax -> matmul fused in one kernel).
 //
 // B200 mapping (one CTA = 256 query rows of one (batch, head)):
-//   warp 9       TMA producer: Q tiles once, then a ring of K and V tiles
+//   warp 10      TMA producer: Q tiles once, then a ring of K and V tiles
 //                (128 keys x d each, 128-byte swizzle) with mbarrier hand-off.
-//   warp 8       tcgen05 issuer (one thread): S_t = Q_t K_j^T into tensor
-//                memory (fp32), then O_t += P_t V_j with P_t read from tensor
-//                memory.  Two query tiles t = 0, 1 alternate so the tensor
-//                core works on one tile while the other tile's softmax runs.
+//   warps 8, 9   tcgen05 issuers: warp 8 issues S_t = Q_t K_j^T into tensor
+//                memory (fp32), warp 9 issues O_t += P_t V_j with P_t read from
+//                tensor memory.  Two query tiles t = 0, 1 alternate so the
+//                tensor core works on one tile while the other tile's softmax
+//                runs.
 //   warps 0-3/4-7 softmax warpgroup of tile 0/1: thread r owns row r of its
 //                tile (tensor-memory lane r), so row max and row sum are
 //                in-thread; it masks boundary tiles, keeps the running max m
@@ -54,7 +55,7 @@ struct FwdCfg {
   static constexpr int kChunk = 128 * 64 * 2;       // one 128-row x 64-column swizzled chunk
   static constexpr int kTileBytes = 128 * D * 2;    // a 128-row tile
   static constexpr int kStages = D == 64 ? 4 : 2;   // K ring and V ring depth
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;
   static constexpr int kSmemQ = 1024;
   static constexpr int kSmemK = kSmemQ + kTiles * kTileBytes;
   static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
@@ -118,7 +119,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Cfg = FwdCfg<D>;
@@ -133,8 +134,7 @@ __global__ void __launch_bounds__(320, 1)
   // barrier block at the head of shared memory
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
   const uint32_t bar_q = smem_u32(&bars[0]);
-  auto bar_kfull = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto bar_vfull = [&](int s) { return smem_u32(&bars[1 + S + s]); };
+  auto bar_kvfull = [&](int s) { return smem_u32(&bars[1 + s]); };  // K_j and V_j landed
   auto bar_kempty = [&](int s) { return smem_u32(&bars[1 + 2 * S + s]); };
   auto bar_vempty = [&](int s) { return smem_u32(&bars[1 + 3 * S + s]); };
   auto bar_sfull = [&](int t) { return smem_u32(&bars[1 + 4 * S + t]); };
@@ -183,8 +183,7 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar_kfull(s), 1);
-      mbar_init(bar_vfull(s), 1);
+      mbar_init(bar_kvfull(s), 1);
       mbar_init(bar_kempty(s), 1);
       mbar_init(bar_vempty(s), 1);
     }
@@ -208,7 +207,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 9) {
+  if (warp == 10) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && JHI > JLO) {
       tma_prefetch_desc(&tmQ);
@@ -222,31 +221,32 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int j = JLO; j < JHI && ok; ++j) {
         const int idx = j - JLO, s = idx % S, u = idx / S;
-        if (u > 0) ok = mbar_wait(bar_kempty(s), (u - 1) & 1, wc);
+        if (u > 0) {  // both readers of the stage are done: S(j - S) and P V(j - S)
+          ok = mbar_wait(bar_kempty(s), (u - 1) & 1, wc);
+          if (ok) ok = mbar_wait(bar_vempty(s), (u - 1) & 1, wc);
+        }
         if (!ok) break;
-        mbar_arrive_expect_tx(bar_kfull(s), Cfg::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
+        mbar_arrive_expect_tx(bar_kvfull(s), 2 * Cfg::kTileBytes);
+        for (int c = 0; c < D / 64; ++c) {
           tma_load_4d(sbase + Cfg::kSmemK + s * Cfg::kTileBytes + c * Cfg::kChunk, &tmK,
-                      bar_kfull(s), c * 64, j * 128, g, b);
-        if (u > 0) ok = mbar_wait(bar_vempty(s), (u - 1) & 1, wc);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar_vfull(s), Cfg::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
+                      bar_kvfull(s), c * 64, j * 128, g, b);
           tma_load_4d(sbase + Cfg::kSmemV + s * Cfg::kTileBytes + c * Cfg::kChunk, &tmV,
-                      bar_vfull(s), c * 64, j * 128, g, b);
+                      bar_kvfull(s), c * 64, j * 128, g, b);
+        }
       }
     }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs this loop and waits; one elected lane issues each
-    // batch of MMAs and its commit.
+  } else if (warp == 8 || warp == 9) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 8 issues S_t = Q_t K^T, warp 9 issues O_t += P_t V.  An MMA issue
+    // blocks until the tensor pipe accepts it, so one issuing warp would leave
+    // the pipe idle during each of its barrier waits; with two, one warp's
+    // waits overlap the other warp's MMAs.  Each warp runs its loop converged
+    // and one elected lane issues each batch and its commits (tcgen05.commit
+    // covers the MMAs of the committing thread).
     if (JHI > JLO) {
-      const uint32_t idesc_qk = make_idesc_f16(BF16, 128, 128, false, false) | (p.qk_negate << 13);
-      const uint32_t idesc_pv = make_idesc_f16(BF16, 128, D, false, true);
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
       };
-      bool ok = wait_all(bar_q, 0);
       auto in_range = [&](int t, int j) {
         return t ? (j >= jlo1 && j < jhi1) : (j >= jlo0 && j < jhi0);
       };
@@ -254,94 +254,156 @@ __global__ void __launch_bounds__(320, 1)
       // (address >> 4) to them
       constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
       constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // V, MN-major
-      const uint64_t dQ0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
-      const uint64_t dK0 = sdesc_at(kDescK, sbase + Cfg::kSmemK);
-      const uint64_t dV0 = sdesc_at(kDescMN, sbase + Cfg::kSmemV);
-      auto issue_s = [&](int t, int j) -> bool {
-        const int idx = j - JLO, s = idx % S, u = idx / S;
-        if (!wait_all(bar_kfull(s), u & 1)) return false;
-        tc_fence_after();
-        const uint64_t qa = dQ0 + uint64_t((t * Cfg::kTileBytes) >> 4);
-        const uint64_t kb = dK0 + uint64_t((s * Cfg::kTileBytes) >> 4);
-        const uint32_t dst = tmem + t * 128;
-        if (elect_one()) {
+      bool ok = true;
+      if constexpr (!kSepP) {
+        // P_t overlays S_t (d = 128): one warp issues everything, so S_t(j+1)
+        // follows P_t V_j in the in-order tensor pipe without waiting for it
+        if (warp == 8) {
+          const uint32_t idesc_qk =
+              make_idesc_f16(BF16, 128, 128, false, false) | (p.qk_negate << 13);
+          const uint32_t idesc_pv = make_idesc_f16(BF16, 128, D, false, true);
+          const uint64_t dQ0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
+          const uint64_t dK0 = sdesc_at(kDescK, sbase + Cfg::kSmemK);
+          const uint64_t dV0 = sdesc_at(kDescMN, sbase + Cfg::kSmemV);
+          auto issue_s = [&](int t, int j) {
+            const int s = (j - JLO) % S;
+            const uint64_t qa = dQ0 + uint64_t((t * Cfg::kTileBytes) >> 4);
+            const uint64_t kb = dK0 + uint64_t((s * Cfg::kTileBytes) >> 4);
+            if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(dst, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_sfull(t));
-        }
-        __syncwarp();
-        return true;
-      };
-      auto issue_pv = [&](int t, int j, int s) {
-        const int jlo_t = t ? jlo1 : jlo0;
-        const uint32_t pbase = kSepP ? tmem + Cfg::kColP + t * 64 : tmem + t * 128;
-        const uint32_t dst = tmem + Cfg::kColO + t * D;
-        const uint64_t vb = dV0 + uint64_t((s * Cfg::kTileBytes) >> 4);
-        const uint32_t acc0 = j > jlo_t ? 1u : 0u;
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            // P_t: 16 keys of 16-bit values = 8 tensor-memory columns per step
-            mma_ts(dst, pbase + kk * 8, vb + uint64_t((kk * 16 * 128) >> 4), idesc_pv,
-                   kk > 0 ? 1u : acc0);
-          }
-          mma_commit(bar_odone(t));
-        }
-        __syncwarp();
-      };
-      for (int t = 0; t < 2 && ok; ++t)
-        if (in_range(t, JLO)) ok = issue_s(t, JLO);
-      for (int j = JLO; j < JHI && ok; ++j) {
-        const int idx = j - JLO, s = idx % S, u = idx / S;
-        bool v_ready = false;
-        if constexpr (kSepP) {
-          // S_t(j+1) as soon as the softmax has read S_t(j); then the P V products
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (!in_range(t, j + 1)) continue;
-            if (in_range(t, j)) {
-              const int jlo_t = t ? jlo1 : jlo0;
-              ok = wait_all(bar_sfree(t), (j - jlo_t) & 1);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t off = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+                mma_ss(tmem + t * 128, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(bar_sfull(t));
             }
-            if (ok) ok = issue_s(t, j + 1);
+            __syncwarp();
+          };
+          auto issue_pv = [&](int t, int j) {
+            const int s = (j - JLO) % S;
+            const int jlo_t = t ? jlo1 : jlo0;
+            const uint64_t vb = dV0 + uint64_t((s * Cfg::kTileBytes) >> 4);
+            const uint32_t acc0 = j > jlo_t ? 1u : 0u;
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < 128 / 16; ++kk)
+                mma_ts(tmem + Cfg::kColO + t * D, tmem + t * 128 + kk * 8,
+                       vb + uint64_t((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+              mma_commit(bar_odone(t));
+            }
+            __syncwarp();
+          };
+          ok = wait_all(bar_q, 0);
+          if (ok) ok = wait_all(bar_kvfull(0), 0);
+          if (ok) {
+            tc_fence_after();
+            for (int t = 0; t < 2; ++t)
+              if (in_range(t, JLO)) issue_s(t, JLO);
           }
+          for (int j = JLO; j < JHI && ok; ++j) {
+            const int idx = j - JLO, s = idx % S;
+            const int s1 = (idx + 1) % S, u1 = (idx + 1) / S;
+            bool next_ready = false;
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (in_range(t, j)) {
+                const int jlo_t = t ? jlo1 : jlo0;
+                if (!(ok = wait_all(bar_pfull(t), (j - jlo_t) & 1))) break;
+                tc_fence_after();
+                issue_pv(t, j);
+              }
+              if (in_range(t, j + 1)) {
+                if (!next_ready) {
+                  if (!(ok = wait_all(bar_kvfull(s1), u1 & 1))) break;
+                  next_ready = true;
+                }
+                tc_fence_after();
+                issue_s(t, j + 1);
+              }
+            }
+            if (!ok) break;
+            if (elect_one()) {
+              mma_commit(bar_kempty(s));
+              mma_commit(bar_vempty(s));
+            }
+            __syncwarp();
+          }
+        }
+      } else if (warp == 8) {
+        const uint32_t idesc_qk =
+            make_idesc_f16(BF16, 128, 128, false, false) | (p.qk_negate << 13);
+        const uint64_t dQ0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
+        const uint64_t dK0 = sdesc_at(kDescK, sbase + Cfg::kSmemK);
+        ok = wait_all(bar_q, 0);
+        for (int j = JLO; j < JHI && ok; ++j) {
+          const int idx = j - JLO, s = idx % S, u = idx / S;
+          bool kv_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (!in_range(t, j)) continue;
-            if (!v_ready) {
-              ok = wait_all(bar_vfull(s), u & 1);
-              v_ready = true;
-            }
-            const int jlo_t = t ? jlo1 : jlo0;
-            if (ok) ok = wait_all(bar_pfull(t), (j - jlo_t) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, j, s);
-          }
-        } else {
-          // P_t aliases S_t: S_t(j+1) follows P_t V_j in the tensor pipe
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (in_range(t, j)) {
-              if (!v_ready) {
-                ok = wait_all(bar_vfull(s), u & 1);
-                v_ready = true;
-              }
-              const int jlo_t = t ? jlo1 : jlo0;
-              if (ok) ok = wait_all(bar_pfull(t), (j - jlo_t) & 1);
+            if (j > (t ? jlo1 : jlo0)) {
+              // the softmax must be done with S_t(j-1): read it (separate P) or
+              // had P_t(j-1) V consumed (P over S)
+              const int prev = j - 1 - (t ? jlo1 : jlo0);
+              ok = kSepP ? wait_all(bar_sfree(t), prev & 1) : wait_all(bar_odone(t), prev & 1);
               if (!ok) break;
-              tc_fence_after();
-              issue_pv(t, j, s);
             }
-            if (ok && in_range(t, j + 1)) ok = issue_s(t, j + 1);
+            if (!kv_ready) {
+              ok = wait_all(bar_kvfull(s), u & 1);
+              kv_ready = true;
+              if (!ok) break;
+            }
+            tc_fence_after();
+            const uint64_t qa = dQ0 + uint64_t((t * Cfg::kTileBytes) >> 4);
+            const uint64_t kb = dK0 + uint64_t((s * Cfg::kTileBytes) >> 4);
+            const uint32_t dst = tmem + t * 128;
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t off = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+                mma_ss(dst, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(bar_sfull(t));
+            }
+            __syncwarp();
           }
+          if (!ok) break;
+          if (elect_one()) mma_commit(bar_kempty(s));  // K_j: both S_t(j) issued
+          __syncwarp();
         }
-        if (!ok) break;
-        if (elect_one()) {
-          mma_commit(bar_kempty(s));
-          mma_commit(bar_vempty(s));
+      } else {
+        const uint32_t idesc_pv = make_idesc_f16(BF16, 128, D, false, true);
+        const uint64_t dV0 = sdesc_at(kDescMN, sbase + Cfg::kSmemV);
+        for (int j = JLO; j < JHI && ok; ++j) {
+          const int idx = j - JLO, s = idx % S, u = idx / S;
+          bool kv_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!in_range(t, j)) continue;
+            const int jlo_t = t ? jlo1 : jlo0;
+            if (!kv_ready) {
+              ok = wait_all(bar_kvfull(s), u & 1);
+              kv_ready = true;
+              if (!ok) break;
+            }
+            if (!(ok = wait_all(bar_pfull(t), (j - jlo_t) & 1))) break;
+            tc_fence_after();
+            const uint32_t pbase = kSepP ? tmem + Cfg::kColP + t * 64 : tmem + t * 128;
+            const uint32_t dst = tmem + Cfg::kColO + t * D;
+            const uint64_t vb = dV0 + uint64_t((s * Cfg::kTileBytes) >> 4);
+            const uint32_t acc0 = j > jlo_t ? 1u : 0u;
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < 128 / 16; ++kk) {
+                // P_t: 16 keys of 16-bit values = 8 tensor-memory columns per step
+                mma_ts(dst, pbase + kk * 8, vb + uint64_t((kk * 16 * 128) >> 4), idesc_pv,
+                       kk > 0 ? 1u : acc0);
+              }
+              mma_commit(bar_odone(t));
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          if (elect_one()) mma_commit(bar_vempty(s));  // V_j: both P_t V_j issued
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
   } else {
