@@ -65,7 +65,13 @@ struct FwdCfg {
   static constexpr bool kSepP = D == 64;            // P in its own tensor-memory region
   static constexpr uint32_t kColP = 384;            // P_t at 384 + 64 t (d = 64 only)
   // of every 8 column pairs of a row, how many take the FMA-pipe exp2
-  static constexpr int kEmuPairsPer8 = D == 64 ? 3 : 1;
+#ifndef FA_FWD_EMU_PAIRS_D64  // tuning overrides (compile-time)
+#define FA_FWD_EMU_PAIRS_D64 3
+#endif
+#ifndef FA_FWD_EMU_PAIRS_D128
+#define FA_FWD_EMU_PAIRS_D128 0
+#endif
+  static constexpr int kEmuPairsPer8 = D == 64 ? FA_FWD_EMU_PAIRS_D64 : FA_FWD_EMU_PAIRS_D128;
 };
 
 // Visible key range of query row i, [lo, hi] inclusive; empty if lo > hi.
@@ -80,8 +86,8 @@ __device__ __forceinline__ void row_key_range(int i, int Nq, int Nk, int causal,
 // ---------------------------------------------------------------- exp2 on the FMA pipe
 // 2^x for a pair: x = n + f with n = round(x) (the 1.5 * 2^23 addition rounds
 // to an integer in the low mantissa bits), f in [-1/2, 1/2]; 2^f by a minimax
-// polynomial (relative error 2.7e-6 at degree 4, 7.5e-5 at degree 3, see
-// fit_exp2_poly.py); 2^n built directly in the exponent field.  x is clamped
+// polynomial of degree 3 (relative error 7.5e-5, see fit_exp2_poly.py); 2^n
+// built directly in the exponent field.  x is clamped
 // at -127 first, where the exponent field becomes 0 and the result is +0, so
 // masked (-inf) scores give exactly 0.
 template <bool BF16>
@@ -92,19 +98,12 @@ __device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
   const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
   const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
   const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-  float2 p;
-  if constexpr (BF16) {  // degree 3: far below bf16 rounding of P
-    p = __ffma2_rn(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
-                   make_float2(2.426111251e-01f, 2.426111251e-01f));
-    p = __ffma2_rn(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
-    p = __ffma2_rn(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
-  } else {  // degree 4: below fp16 rounding of P
-    p = __ffma2_rn(make_float2(9.570102207e-03f, 9.570102207e-03f), f,
-                   make_float2(5.591785908e-02f, 5.591785908e-02f));
-    p = __ffma2_rn(p, f, make_float2(2.402474433e-01f, 2.402474433e-01f));
-    p = __ffma2_rn(p, f, make_float2(6.931217909e-01f, 6.931217909e-01f));
-    p = __ffma2_rn(p, f, make_float2(9.999992847e-01f, 9.999992847e-01f));
-  }
+  // degree 3 (relative error 7.5e-5): below the rounding of P to bf16 (2^-9)
+  // and to fp16 (2^-12, 6.5x larger)
+  float2 p = __ffma2_rn(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
+                        make_float2(2.426111251e-01f, 2.426111251e-01f));
+  p = __ffma2_rn(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+  p = __ffma2_rn(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
   // (n + 127) << 23: the low bits of t hold n + 2^22 + 2^23, whose shifted-out
   // high part vanishes modulo 2^32
   const float sx = __uint_as_float((__float_as_uint(t.x) << 23) + (127u << 23));
