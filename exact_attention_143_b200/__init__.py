@@ -36,7 +36,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
-            "fa_bwd_noalloc")
+            "fa_bwd_noalloc", "fa_selftest_wait_timeout")
 
 _lib = None
 
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_set_bwd_main_events.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [i64p] * 8 + [i, f, i, i, i, vp]
     lib.fa_bwd_noalloc.restype = i
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.fa_selftest_wait_timeout.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -200,6 +202,18 @@ def set_bwd_main_events(start=None, stop=None) -> None:
     h0 = ctypes.c_void_p(start.cuda_event) if start is not None else None
     h1 = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
     lib.fa_set_bwd_main_events(h0, h1)
+
+
+def selftest_wait_timeout(limit_ns: int, device=None) -> int:
+    """Launch the bounded-wait self-test kernel (see include/fa143.h) and
+    return fa_get_device_error()'s status afterwards."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        rc = lib.fa_selftest_wait_timeout(int(limit_ns), _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_selftest_wait_timeout")
+    return get_device_error(dev)
 
 
 def set_wait_limit_ns(limit_ns: int) -> int:

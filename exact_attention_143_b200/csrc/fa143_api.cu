@@ -137,6 +137,23 @@ float scale_log2_of(float scale) {
   return a > 0.f ? a : 1e-30f;
 }
 
+// A wait on a barrier nothing completes: exercises the timeout path of the
+// bounded waits (error word set, kernel returns) without any copy in flight.
+__global__ void fa_selftest_wait_kernel(unsigned int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(fa::smem_u32(&bar), 1);
+    abort_flag = 0;
+    fa::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    fa::WaitCtx wc{&abort_flag, err, limit_ns};
+    fa::mbar_wait(fa::smem_u32(&bar), 0, wc);
+  }
+}
+
 template <int D, bool BF16>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const fa::FwdParams& prm, cudaStream_t st) {
@@ -205,6 +222,14 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     default: return "unknown status";
   }
+}
+
+int fa_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return FA_ERR_INVALID_ARG;
+  unsigned int* err = device_error_ptr();
+  if (!err) return FA_ERR_CUDA;
+  fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_set_bwd_main_events(void* ev_start, void* ev_stop) {

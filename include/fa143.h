@@ -176,6 +176,18 @@ int fa_get_device_error(void* stream);
 int fa_set_bwd_main_events(void* ev_start, void* ev_stop);
 
 /*
+ * Self-test of the bounded device-side waits.  Launches one small kernel on
+ * `stream` whose thread waits, through the same bounded wait the attention
+ * kernels use, on a shared-memory barrier that nothing ever completes.  After
+ * limit_ns the wait gives up, records FA_ERR_DEVICE_TIMEOUT in the device
+ * error word and the kernel returns; no copy or tensor-core operation is in
+ * flight, so the context stays usable.  Read the outcome with
+ * fa_get_device_error().  Returns FA_OK once launched, FA_ERR_INVALID_ARG if
+ * limit_ns is 0 or above 10 s.
+ */
+int fa_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
  * Sets the per-wait limit of device-side waits, in nanoseconds (default
  * 2e9).  Returns the previous value.  For tests of the timeout path only.
  */
