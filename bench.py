@@ -37,7 +37,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from seeded_inputs import WORKLOADS, Workload, make_qkv, make_workload_inputs  # noqa: E402
+from seeded_inputs import (VARLEN_WORKLOADS, WORKLOADS, Workload, make_qkv,  # noqa: E402
+                           make_varlen_inputs, make_workload_inputs)
 
 METRIC = "attention TFLOPS (fwd, fwd+bwd) on 1 B200 and % of dense FP16/BF16 tensor peak"
 MAIN_WORKLOAD = "fwdbwd_1x16384_h16_d128_bf16_causal"
@@ -356,6 +357,29 @@ def run_ours(args):
             table[name] = {"fwd_ms_median": round(med, 4), "fwd_ms_min": round(min(tms), 4),
                            "fwd_tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
             del tq, tk, tv, to, tl
+        # packed variable-length batch (no padding): forward and backward
+        for vw in VARLEN_WORKLOADS.values():
+            vq, vk, vv, vdo, vcu, lens = make_varlen_inputs(vw)
+            vq, vk, vv, vdo, vcu = (t.to(dev) for t in (vq, vk, vv, vdo, vcu))
+            mx = max(lens)
+            vkw = dict(softmax_scale=vw.softmax_scale, causal=vw.causal)
+            vo, vl = fa.fa_fwd_varlen(vq, vk, vv, vcu, vcu, mx, mx, **vkw)
+            vws = torch.empty(fa.bwd_workspace_size(len(lens), mx, vw.q_heads, vw.head_dim),
+                              dtype=torch.uint8, device=dev)
+            vdq, vdk, vdv = torch.empty_like(vq), torch.empty_like(vk), torch.empty_like(vv)
+            vf = sum(4.0 * vw.q_heads * vw.head_dim * visible_pairs(n, n, vw.causal, (-1, -1))
+                     for n in lens)
+            fms_v = time_steps(lambda _: fa.fa_fwd_varlen(vq, vk, vv, vcu, vcu, mx, mx, out=vo,
+                                                          lse=vl, **vkw), 10, 3, flush, stream)
+            bms_v = time_steps(lambda _: fa.fa_bwd_varlen(vdo, vq, vk, vv, vo, vl, vcu, vcu, mx, mx,
+                                                          dq=vdq, dk=vdk, dv=vdv, workspace=vws,
+                                                          **vkw), 10, 3, flush, stream)
+            fm_v, bm_v = statistics.median(fms_v), statistics.median(bms_v)
+            table[vw.name] = {"total_tokens": sum(lens), "fwd_ms_median": round(fm_v, 4),
+                              "fwd_tflops": round(vf / (fm_v / 1e3) / 1e12, 1),
+                              "bwd_ms_median": round(bm_v, 4),
+                              "bwd_tflops": round(2.5 * vf / (bm_v / 1e3) / 1e12, 1)}
+            del vq, vk, vv, vdo, vo, vl, vws, vdq, vdk, vdv
         # the main workload's forward and backward separately
         fms = time_steps(lambda _: fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw), 10, 3, flush,
                          stream)

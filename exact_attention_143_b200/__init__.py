@@ -36,7 +36,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
-            "fa_bwd_noalloc", "fa_selftest_wait_timeout")
+            "fa_bwd_noalloc", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen")
 
 _lib = None
 
@@ -75,6 +75,11 @@ def load_library(path: str = LIB_PATH):
     lib.fa_set_bwd_main_events.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [i64p] * 8 + [i, f, i, i, i, vp]
     lib.fa_bwd_noalloc.restype = i
+    lib.fa_fwd_varlen.argtypes = [vp] * 7 + [i] * 8 + [i64p] * 4 + [i, f, i, i, i, vp]
+    lib.fa_fwd_varlen.restype = i
+    lib.fa_bwd_varlen.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [vp, vp] + [i] * 8 +
+                                  [i64p] * 8 + [i, f, i, i, i, vp])
+    lib.fa_bwd_varlen.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.fa_selftest_wait_timeout.restype = i
     if path == LIB_PATH:
@@ -146,6 +151,94 @@ def fa_fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), out=
     if rc:
         raise FAError(rc, "fa_fwd")
     return out, lse
+
+
+def _strides2(t: torch.Tensor):
+    if t.dim() != 3:
+        raise ValueError("expected a packed [tokens, heads, head_dim] tensor, got shape %s"
+                         % (tuple(t.shape),))
+    if t.stride(2) != 1 and t.shape[2] > 1:
+        raise ValueError("head_dim must be contiguous (stride 1)")
+    return (ctypes.c_int64 * 2)(t.stride(0), t.stride(1))
+
+
+def _check_cu(cu, n):
+    if cu.dtype != torch.int32 or not cu.is_cuda or cu.dim() != 1 or cu.numel() != n + 1 \
+            or not cu.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 CUDA tensor of B + 1 offsets")
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                  softmax_scale=None, causal=False, window_size=(-1, -1), out=None, lse=None):
+    """Forward over a packed variable-length batch (no padding).
+
+    q [total_q, Hq, d], k/v [total_k, Hkv, d]; cu_seqlens_q/k int32 [B+1] on the
+    device.  Returns (o [total_q, Hq, d], lse [Hq, total_q] fp32)."""
+    lib = load_library()
+    dev = _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    code = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    _check_cu(cu_seqlens_q, B)
+    _check_cu(cu_seqlens_k, B)
+    if out is None:
+        out = torch.empty((total_q, Hq, d), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=dev)
+    wl, wr = window_size
+    with torch.cuda.device(dev):
+        rc = lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+                               B, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, Hq,
+                               Hkv, d, _strides2(q), _strides2(k), _strides2(v), _strides2(out),
+                               code, _scale(softmax_scale, d), int(bool(causal)), int(wl),
+                               int(wr), _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_fwd_varlen")
+    return out, lse
+
+
+def fa_bwd_varlen(dout, q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                  max_seqlen_k, softmax_scale=None, causal=False, window_size=(-1, -1),
+                  dq=None, dk=None, dv=None, workspace=None):
+    """Backward over a packed variable-length batch; returns (dq, dk, dv)."""
+    lib = load_library()
+    dev = _check_cuda(dout, q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k)
+    code = _dtype_code(q)
+    for t in (k, v, o, dout):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, o, dout must share one dtype")
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    _check_cu(cu_seqlens_q, B)
+    _check_cu(cu_seqlens_k, B)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (Hq, total_q):
+        raise ValueError("lse must be the contiguous fp32 [Hq, total_q] tensor from fa_fwd_varlen")
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(B, int(max_seqlen_q), Hq, d), dtype=torch.uint8,
+                                device=dev)
+    wl, wr = window_size
+    with torch.cuda.device(dev):
+        rc = lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(),
+                               cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B,
+                               int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, Hq, Hkv, d,
+                               _strides2(q), _strides2(k), _strides2(v), _strides2(o),
+                               _strides2(dout), _strides2(dq), _strides2(dk), _strides2(dv),
+                               code, _scale(softmax_scale, d), int(bool(causal)), int(wl),
+                               int(wr), _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_bwd_varlen")
+    return dq, dk, dv
 
 
 def bwd_workspace_size(B, Nq, Hq, d) -> int:

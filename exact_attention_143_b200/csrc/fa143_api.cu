@@ -244,21 +244,22 @@ uint64_t fa_set_wait_limit_ns(uint64_t limit_ns) {
   return old;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
-           int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3], const int64_t k_stride[3],
-           const int64_t v_stride[3], const int64_t o_stride[3], int dtype, float softmax_scale,
-           int causal, int window_left, int window_right, void* stream) {
-  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
-  if (rc) return rc;
-  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
-  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
-  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
-  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
-  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+}  // extern "C"
+
+namespace {
+
+// Shared body of fa_fwd and fa_fwd_varlen.  Dense: tq/tk/tv/to span [B, N, H, d],
+// cu_q == cu_k == nullptr.  Varlen: the descriptors span [1, total, H, d] and
+// B counts the sequences; Nq / Nk are the longest sequence lengths.
+int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
+             const TensorDesc& to, float* lse, size_t lse_bytes, int B, int Nq, int Nk, int Hq,
+             int Hkv, int d, const int* cu_q, const int* cu_k, int total_q, int total_k,
+             int dtype, float softmax_scale, int causal, int window_left, int window_right,
+             void* stream) {
+  int rc;
   for (const TensorDesc* t : {&tq, &tk, &tv, &to})
     if ((rc = check_tensor(*t))) return rc;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_ALIGNMENT;
-  const size_t lse_bytes = size_t(B) * Hq * Nq * sizeof(float);
   if (overlaps_t(to, tq) || overlaps_t(to, tk) || overlaps_t(to, tv) ||
       overlaps_span(tq, lse, lse_bytes) || overlaps_span(tk, lse, lse_bytes) ||
       overlaps_span(tv, lse, lse_bytes) || overlaps_span(to, lse, lse_bytes))
@@ -269,11 +270,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
       (rc = make_map(&mv, tv, dtype)))
     return rc;
   fa::FwdParams prm{};
-  prm.o = o;
+  prm.o = const_cast<void*>(to.ptr);
   prm.lse = lse;
-  prm.o_sb = o_stride[0];
-  prm.o_ss = o_stride[1];
-  prm.o_sh = o_stride[2];
+  prm.o_sb = to.sb;
+  prm.o_ss = to.ss;
+  prm.o_sh = to.sh;
   prm.B = B;
   prm.Nq = Nq;
   prm.Nk = Nk;
@@ -287,6 +288,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   prm.wr = window_right;
   prm.err = device_error_ptr();
   prm.wait_limit_ns = g_wait_limit_ns;
+  prm.cu_q = cu_q;
+  prm.cu_k = cu_k;
+  prm.total_q = total_q;
+  prm.total_k = total_k;
   if (!prm.err) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16)
@@ -296,39 +301,85 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
                  : launch_fwd<128, false>(mq, mk, mv, prm, st);
 }
 
+int check_varlen(const int* cu_q, const int* cu_k, int B, int max_q, int max_k, int total_q,
+                 int total_k) {
+  if (!cu_q || !cu_k) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_k) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (B < 1 || max_q < 1 || max_k < 1 || total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
+  if (max_q > total_q || max_k > total_k) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+           int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3], const int64_t k_stride[3],
+           const int64_t v_stride[3], const int64_t o_stride[3], int dtype, float softmax_scale,
+           int causal, int window_left, int window_right, void* stream) {
+  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  if (rc) return rc;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  return fwd_impl(tq, tk, tv, to, lse, size_t(B) * Hq * Nq * sizeof(float), B, Nq, Nk, Hq, Hkv,
+                  d, nullptr, nullptr, 0, 0, dtype, softmax_scale, causal, window_left,
+                  window_right, stream);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d,
+                  const int64_t q_stride[2], const int64_t k_stride[2],
+                  const int64_t v_stride[2], const int64_t o_stride[2], int dtype,
+                  float softmax_scale, int causal, int window_left, int window_right,
+                  void* stream) {
+  int rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale,
+                        window_left, window_right);
+  if (rc) return rc;
+  if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
+                         total_k)))
+    return rc;
+  if (total_q > (1 << 28) || total_k > (1 << 28)) return FA_ERR_INVALID_ARG;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, 0, q_stride[0], q_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tk{k, 0, k_stride[0], k_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc tv{v, 0, v_stride[0], v_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
+  return fwd_impl(tq, tk, tv, to, lse, size_t(Hq) * total_q * sizeof(float), B, max_seqlen_q,
+                  max_seqlen_k, Hq, Hkv, d, cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype,
+                  softmax_scale, causal, window_left, window_right, stream);
+}
+
 size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d) {
   if (B < 1 || Nq < 1 || Hq < 1 || d < 1) return 0;
   const size_t nq_pad = (size_t(Nq) + 127) / 128 * 128;
   return (size_t(B) * Hq * Nq * d + 2 * size_t(B) * Hq * nq_pad) * sizeof(float);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-           const float* lse, void* dq, void* dk, void* dv, void* workspace,
-           size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
-           const int64_t q_stride[3], const int64_t k_stride[3], const int64_t v_stride[3],
-           const int64_t o_stride[3], const int64_t do_stride[3], const int64_t dq_stride[3],
-           const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
-           float softmax_scale, int causal, int window_left, int window_right, void* stream) {
-  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
-  if (rc) return rc;
-  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
-      !dk_stride || !dv_stride || !lse)
-    return FA_ERR_INVALID_ARG;
-  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
-  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
-  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
-  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
-  const TensorDesc tdo{dout, do_stride[0], do_stride[1], do_stride[2], B, Nq, Hq, d};
-  const TensorDesc tdq{dq, dq_stride[0], dq_stride[1], dq_stride[2], B, Nq, Hq, d};
-  const TensorDesc tdk{dk, dk_stride[0], dk_stride[1], dk_stride[2], B, Nk, Hkv, d};
-  const TensorDesc tdv{dv, dv_stride[0], dv_stride[1], dv_stride[2], B, Nk, Hkv, d};
+}  // extern "C"
+
+namespace {
+
+// Shared body of fa_bwd and fa_bwd_varlen (see fwd_impl for the conventions).
+int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
+             const TensorDesc& to, const TensorDesc& tdo, const TensorDesc& tdq,
+             const TensorDesc& tdk, const TensorDesc& tdv, const float* lse, size_t lse_bytes,
+             void* workspace, size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv,
+             int d, const int* cu_q, const int* cu_k, int total_q, int total_k, int dtype,
+             float softmax_scale, int causal, int window_left, int window_right, void* stream) {
+  int rc;
   for (const TensorDesc* t : {&tq, &tk, &tv, &to, &tdo, &tdq, &tdk, &tdv})
     if ((rc = check_tensor(*t))) return rc;
+  if (!lse) return FA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_ALIGNMENT;
   const size_t need = fa_bwd_workspace_size(B, Nq, Hq, d);
   if (workspace == nullptr || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
-  const size_t lse_bytes = size_t(B) * Hq * Nq * sizeof(float);
   // outputs (dq, dk, dv, workspace) must not overlap each other or any input
   const TensorDesc* ins[] = {&tq, &tk, &tv, &to, &tdo};
   const TensorDesc* outs[] = {&tdq, &tdk, &tdv};
@@ -362,24 +413,26 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   const bool bf16 = dtype == FA_BF16;
 
   fa::BwdPrepParams pp{};
-  pp.o = o;
-  pp.dout = dout;
+  pp.o = to.ptr;
+  pp.dout = tdo.ptr;
   pp.lse = lse;
   pp.lse2 = lse2;
   pp.Dvec = Dvec;
   pp.dq_acc = reinterpret_cast<float4*>(dq_acc);
-  pp.o_sb = o_stride[0];
-  pp.o_ss = o_stride[1];
-  pp.o_sh = o_stride[2];
-  pp.do_sb = do_stride[0];
-  pp.do_ss = do_stride[1];
-  pp.do_sh = do_stride[2];
+  pp.o_sb = to.sb;
+  pp.o_ss = to.ss;
+  pp.o_sh = to.sh;
+  pp.do_sb = tdo.sb;
+  pp.do_ss = tdo.ss;
+  pp.do_sh = tdo.sh;
   pp.B = B;
   pp.Nq = Nq;
   pp.Nq_pad = nq_pad;
   pp.Hq = Hq;
   pp.d = d;
   pp.dq_acc_vec4 = int64_t(B) * Hq * Nq * d / 4;
+  pp.cu_q = cu_q;
+  pp.total_q = total_q;
   {
     const int64_t rows = int64_t(B) * Hq * nq_pad;
     const int64_t blocks = std::min<int64_t>((rows + 7) / 8, 148 * 16);
@@ -394,14 +447,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   bp.lse2 = lse2;
   bp.Dvec = Dvec;
   bp.dq_acc = dq_acc;
-  bp.dk = dk;
-  bp.dv = dv;
-  bp.dk_sb = dk_stride[0];
-  bp.dk_ss = dk_stride[1];
-  bp.dk_sh = dk_stride[2];
-  bp.dv_sb = dv_stride[0];
-  bp.dv_ss = dv_stride[1];
-  bp.dv_sh = dv_stride[2];
+  bp.dk = const_cast<void*>(tdk.ptr);
+  bp.dv = const_cast<void*>(tdv.ptr);
+  bp.dk_sb = tdk.sb;
+  bp.dk_ss = tdk.ss;
+  bp.dk_sh = tdk.sh;
+  bp.dv_sb = tdv.sb;
+  bp.dv_ss = tdv.ss;
+  bp.dv_sh = tdv.sh;
   bp.B = B;
   bp.Nq = Nq;
   bp.Nq_pad = nq_pad;
@@ -416,6 +469,10 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   bp.wr = window_right;
   bp.err = err;
   bp.wait_limit_ns = g_wait_limit_ns;
+  bp.cu_q = cu_q;
+  bp.cu_k = cu_k;
+  bp.total_q = total_q;
+  bp.total_k = total_k;
   if (g_bwd_ev_start && cudaEventRecord(g_bwd_ev_start, st) != cudaSuccess) return FA_ERR_CUDA;
   if (bf16)
     rc = d == 64 ? launch_bwd<64, true>(mq, mk, mv, mdo, bp, st)
@@ -428,14 +485,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
 
   fa::BwdConvertParams cp{};
   cp.dq_acc = dq_acc;
-  cp.dq = dq;
-  cp.dq_sb = dq_stride[0];
-  cp.dq_ss = dq_stride[1];
-  cp.dq_sh = dq_stride[2];
+  cp.dq = const_cast<void*>(tdq.ptr);
+  cp.dq_sb = tdq.sb;
+  cp.dq_ss = tdq.ss;
+  cp.dq_sh = tdq.sh;
   cp.B = B;
   cp.Nq = Nq;
   cp.Hq = Hq;
   cp.d = d;
+  cp.cu_q = cu_q;
+  cp.total_q = total_q;
   {
     const int64_t n = int64_t(B) * Hq * Nq * (d / 8);
     const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 32);
@@ -446,6 +505,69 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, void* workspace,
+           size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+           const int64_t q_stride[3], const int64_t k_stride[3], const int64_t v_stride[3],
+           const int64_t o_stride[3], const int64_t do_stride[3], const int64_t dq_stride[3],
+           const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
+           float softmax_scale, int causal, int window_left, int window_right, void* stream) {
+  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  if (rc) return rc;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
+      !dk_stride || !dv_stride)
+    return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdo{dout, do_stride[0], do_stride[1], do_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdq{dq, dq_stride[0], dq_stride[1], dq_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdk{dk, dk_stride[0], dk_stride[1], dk_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tdv{dv, dv_stride[0], dv_stride[1], dv_stride[2], B, Nk, Hkv, d};
+  return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(B) * Hq * Nq * sizeof(float),
+                  workspace, workspace_bytes, B, Nq, Nk, Hq, Hkv, d, nullptr, nullptr, 0, 0,
+                  dtype, softmax_scale, causal, window_left, window_right, stream);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                  int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq,
+                  int Hkv, int d, const int64_t q_stride[2], const int64_t k_stride[2],
+                  const int64_t v_stride[2], const int64_t o_stride[2],
+                  const int64_t do_stride[2], const int64_t dq_stride[2],
+                  const int64_t dk_stride[2], const int64_t dv_stride[2], int dtype,
+                  float softmax_scale, int causal, int window_left, int window_right,
+                  void* stream) {
+  int rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale,
+                        window_left, window_right);
+  if (rc) return rc;
+  if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
+                         total_k)))
+    return rc;
+  if (total_q > (1 << 28) || total_k > (1 << 28)) return FA_ERR_INVALID_ARG;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
+      !dk_stride || !dv_stride)
+    return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, 0, q_stride[0], q_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tk{k, 0, k_stride[0], k_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc tv{v, 0, v_stride[0], v_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tdo{dout, 0, do_stride[0], do_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tdq{dq, 0, dq_stride[0], dq_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tdk{dk, 0, dk_stride[0], dk_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc tdv{dv, 0, dv_stride[0], dv_stride[1], 1, total_k, Hkv, d};
+  return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(Hq) * total_q * sizeof(float),
+                  workspace, workspace_bytes, B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d,
+                  cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype, softmax_scale, causal,
+                  window_left, window_right, stream);
 }
 
 int fa_get_device_error(void* stream) {

@@ -63,7 +63,22 @@ struct BwdPrepParams {
   int64_t o_sb, o_ss, o_sh, do_sb, do_ss, do_sh;
   int B, Nq, Nq_pad, Hq, d;
   int64_t dq_acc_vec4;  // number of float4 in dq_acc
+  const int* cu_q;      // variable-length batches: token offsets [B + 1] (else nullptr)
+  int total_q;
 };
+
+// Length and first token row of sequence b (dense layout: Nq rows, batch b).
+__device__ __forceinline__ void seq_rows(const int* cu, int b, int total, int maxlen, int& len,
+                                         int& start) {
+  if (cu == nullptr) {
+    len = maxlen;
+    start = 0;
+    return;
+  }
+  const int a0 = min(max(cu[b], 0), total), a1 = min(max(cu[b + 1], a0), total);
+  len = min(a1 - a0, maxlen);
+  start = a0;
+}
 
 template <bool BF16>
 __device__ __forceinline__ float to_f32(uint16_t x) {
@@ -86,13 +101,17 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
     const int64_t bh = r / p.Nq_pad;
     const int h = int(bh % p.Hq), b = int(bh / p.Hq);
     float acc = 0.f, lse2 = INFINITY;
-    if (i < p.Nq) {
-      const uint16_t* orow = static_cast<const uint16_t*>(p.o) + b * p.o_sb + int64_t(i) * p.o_ss +
-                             int64_t(h) * p.o_sh;
-      const uint16_t* drow = static_cast<const uint16_t*>(p.dout) + b * p.do_sb +
-                             int64_t(i) * p.do_ss + int64_t(h) * p.do_sh;
+    int len, start;
+    seq_rows(p.cu_q, b, p.total_q, p.Nq, len, start);
+    const int bc = p.cu_q ? 0 : b;
+    if (i < len) {
+      const uint16_t* orow = static_cast<const uint16_t*>(p.o) + bc * p.o_sb +
+                             int64_t(start + i) * p.o_ss + int64_t(h) * p.o_sh;
+      const uint16_t* drow = static_cast<const uint16_t*>(p.dout) + bc * p.do_sb +
+                             int64_t(start + i) * p.do_ss + int64_t(h) * p.do_sh;
       for (int c = lane; c < p.d; c += 32) acc += to_f32<BF16>(orow[c]) * to_f32<BF16>(drow[c]);
-      const float l = p.lse[(int64_t(b) * p.Hq + h) * p.Nq + i];
+      const float l = p.cu_q ? p.lse[int64_t(h) * p.total_q + start + i]
+                             : p.lse[(int64_t(b) * p.Hq + h) * p.Nq + i];
       lse2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
     }
 #pragma unroll
@@ -114,6 +133,8 @@ struct BwdConvertParams {
   void* dq;
   int64_t dq_sb, dq_ss, dq_sh;
   int B, Nq, Hq, d;
+  const int* cu_q;  // variable-length batches (else nullptr)
+  int total_q;
 };
 
 // One thread per 8 consecutive elements of one row (16-byte store).
@@ -128,6 +149,10 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdConvert
     const int i = int(row % p.Nq);
     const int64_t bh = row / p.Nq;
     const int h = int(bh % p.Hq), b = int(bh / p.Hq);
+    int len, start;
+    seq_rows(p.cu_q, b, p.total_q, p.Nq, len, start);
+    if (i >= len) continue;
+    const int bc = p.cu_q ? 0 : b;
     const float4* src = reinterpret_cast<const float4*>(p.dq_acc + row * p.d + c8 * 8);
     const float4 a = src[0], c = src[1];
     uint4 out;
@@ -135,7 +160,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdConvert
     out.y = pack2<BF16>(a.z, a.w);
     out.z = pack2<BF16>(c.x, c.y);
     out.w = pack2<BF16>(c.z, c.w);
-    uint16_t* dst = static_cast<uint16_t*>(p.dq) + b * p.dq_sb + int64_t(i) * p.dq_ss +
+    uint16_t* dst = static_cast<uint16_t*>(p.dq) + bc * p.dq_sb + int64_t(start + i) * p.dq_ss +
                     int64_t(h) * p.dq_sh + c8 * 8;
     *reinterpret_cast<uint4*>(dst) = out;
   }
@@ -156,6 +181,11 @@ struct BwdParams {
   int causal, wl, wr;
   unsigned int* err;
   uint64_t wait_limit_ns;
+  // variable-length batches: token offsets [B + 1] of q and k (else nullptr);
+  // Nq / Nk then hold the longest sequence lengths
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
 template <int D>
@@ -233,13 +263,19 @@ __global__ void __launch_bounds__(480, 1)
   const int ntile = int(blockIdx.y);
   const int G = p.Hq / p.Hkv;
   const int key0 = ntile * 128;
+  // this sequence's lengths and first rows (dense: the whole tensor, batch b)
+  int Nq, Nk, qstart, kstart;
+  seq_rows(p.cu_q, b, p.total_q, p.Nq, Nq, qstart);
+  seq_rows(p.cu_k, b, p.total_k, p.Nk, Nk, kstart);
+  const int bc = p.cu_q ? 0 : b;
+  if (key0 >= Nk) return;  // no key of this sequence here (CTA-uniform)
 
   // query rows that can see some key of this tile (bounds are monotone in the row)
-  const int off = p.Nk - p.Nq;
+  const int off = Nk - Nq;
   const int right = p.causal ? 0 : p.wr;
-  const int key1 = min(key0 + 127, p.Nk - 1);
+  const int key1 = min(key0 + 127, Nk - 1);
   int i_min = right >= 0 ? max(0, key0 - off - right) : 0;
-  int i_max = p.wl >= 0 ? min(p.Nq - 1, key1 - off + p.wl) : p.Nq - 1;
+  int i_max = p.wl >= 0 ? min(Nq - 1, key1 - off + p.wl) : Nq - 1;
   const int mlo = i_min / 128;
   const int nm = (i_min <= i_max) ? (i_max / 128 - mlo + 1) : 0;
   const int T = nm * G;  // steps: (query head, query tile)
@@ -291,8 +327,10 @@ __global__ void __launch_bounds__(480, 1)
       tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar_kv, 2 * Cfg::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(sbase + Cfg::kSmemK + c * Cfg::kChunk, &tmK, bar_kv, c * 64, key0, g, b);
-        tma_load_4d(sbase + Cfg::kSmemV + c * Cfg::kChunk, &tmV, bar_kv, c * 64, key0, g, b);
+        tma_load_4d(sbase + Cfg::kSmemK + c * Cfg::kChunk, &tmK, bar_kv, c * 64, kstart + key0, g,
+                    bc);
+        tma_load_4d(sbase + Cfg::kSmemV + c * Cfg::kChunk, &tmV, bar_kv, c * 64, kstart + key0, g,
+                    bc);
       }
       for (int s = 0; s < T; ++s) {
         const int st = s & 1, u = s >> 1;
@@ -302,7 +340,7 @@ __global__ void __launch_bounds__(480, 1)
         mbar_arrive_expect_tx(bar_qfull(st), Cfg::kTileBytes + 1024);
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(sbase + Cfg::kSmemQ + st * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ,
-                      bar_qfull(st), c * 64, m * 128, h, b);
+                      bar_qfull(st), c * 64, qstart + m * 128, h, bc);
         const int64_t rowoff = (int64_t(b) * p.Hq + h) * p.Nq_pad + int64_t(m) * 128;
         bulk_load_1d(sbase + Cfg::kSmemLSE + st * 512, p.lse2 + rowoff, 512, bar_qfull(st));
         bulk_load_1d(sbase + Cfg::kSmemDv + st * 512, p.Dvec + rowoff, 512, bar_qfull(st));
@@ -310,8 +348,8 @@ __global__ void __launch_bounds__(480, 1)
         if (s > 0 && !mbar_wait(bar_doempty, (s - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(bar_dofull, Cfg::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sbase + Cfg::kSmemDO + c * Cfg::kChunk, &tmDO, bar_dofull, c * 64, m * 128,
-                      h, b);
+          tma_load_4d(sbase + Cfg::kSmemDO + c * Cfg::kChunk, &tmDO, bar_dofull, c * 64,
+                      qstart + m * 128, h, bc);
       }
     }
   } else if (warp == 14) {
@@ -501,7 +539,7 @@ __global__ void __launch_bounds__(480, 1)
     // queries that see this key: [qlo, qhi]
     int qlo = right >= 0 ? key - off - right : INT_MIN;
     int qhi = p.wl >= 0 ? key - off + p.wl : INT_MAX;
-    if (key >= p.Nk) {
+    if (key >= Nk) {
       qlo = INT_MAX;
       qhi = INT_MIN;
     }
@@ -624,11 +662,11 @@ __global__ void __launch_bounds__(480, 1)
     // dtype; this thread writes half of the columns of key row j
     if (ok) {
       tc_fence_after();
-      const bool store = key < p.Nk;
-      uint16_t* dkrow = static_cast<uint16_t*>(p.dk) + b * p.dk_sb + int64_t(key) * p.dk_ss +
-                        int64_t(g) * p.dk_sh + half * (D / 2);
-      uint16_t* dvrow = static_cast<uint16_t*>(p.dv) + b * p.dv_sb + int64_t(key) * p.dv_ss +
-                        int64_t(g) * p.dv_sh + half * (D / 2);
+      const bool store = key < Nk;
+      uint16_t* dkrow = static_cast<uint16_t*>(p.dk) + bc * p.dk_sb +
+                        int64_t(kstart + key) * p.dk_ss + int64_t(g) * p.dk_sh + half * (D / 2);
+      uint16_t* dvrow = static_cast<uint16_t*>(p.dv) + bc * p.dv_sb +
+                        int64_t(kstart + key) * p.dv_ss + int64_t(g) * p.dv_sh + half * (D / 2);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = (which == 0 ? Cfg::kColDK : Cfg::kColDV) + half * (D / 2);

@@ -47,6 +47,13 @@ struct FwdParams {
   uint32_t qk_negate;        // 1 if softmax_scale < 0 (negate A in Q K^T)
   unsigned int* err;
   uint64_t wait_limit_ns;
+  // variable-length packed batches: sequence b owns token rows
+  // [cu_q[b], cu_q[b+1]) of q/o and [cu_k[b], cu_k[b+1]) of k/v (nullptr for
+  // the dense layout); Nq / Nk then hold the longest sequence lengths and LSE
+  // is [Hq, total_q]
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
 template <int D>
@@ -153,17 +160,29 @@ __global__ void __launch_bounds__(352, 1)
   const int b = bh / p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int mblock = p.n_mblocks - 1 - int(blockIdx.y);
+  // this sequence's lengths and first rows (dense: the whole tensor, batch b)
+  int Nq = p.Nq, Nk = p.Nk, qstart = 0, kstart = 0, bc = b;
+  if (p.cu_q != nullptr) {
+    const int q0 = min(max(p.cu_q[b], 0), p.total_q), q1 = min(max(p.cu_q[b + 1], q0), p.total_q);
+    const int k0 = min(max(p.cu_k[b], 0), p.total_k), k1 = min(max(p.cu_k[b + 1], k0), p.total_k);
+    Nq = min(q1 - q0, p.Nq);
+    Nk = min(k1 - k0, p.Nk);
+    qstart = q0;
+    kstart = k0;
+    bc = 0;
+  }
+  if (mblock * 256 >= Nq) return;  // no query row of this sequence here (CTA-uniform)
 
   // K-tile range [jlo_t, jhi_t) of each query tile t (empty when jlo_t == jhi_t)
   auto tile_range = [&](int t, int& lo_j, int& hi_j) {
     const int r0 = mblock * 256 + t * 128;
     lo_j = 0;
     hi_j = 0;
-    if (r0 < p.Nq) {
-      const int r1 = min(r0 + 127, p.Nq - 1);
+    if (r0 < Nq) {
+      const int r1 = min(r0 + 127, Nq - 1);
       int lo0, hi0, lo1, hi1;
-      row_key_range(r0, p.Nq, p.Nk, p.causal, p.wl, p.wr, lo0, hi0);
-      row_key_range(r1, p.Nq, p.Nk, p.causal, p.wl, p.wr, lo1, hi1);
+      row_key_range(r0, Nq, Nk, p.causal, p.wl, p.wr, lo0, hi0);
+      row_key_range(r1, Nq, Nk, p.causal, p.wl, p.wr, lo1, hi1);
       if (lo0 <= hi1) {  // both bounds grow with the row
         lo_j = lo0 / 128;
         hi_j = hi1 / 128 + 1;
@@ -216,7 +235,7 @@ __global__ void __launch_bounds__(352, 1)
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(sbase + Cfg::kSmemQ + t * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ, bar_q,
-                      c * 64, mblock * 256 + t * 128, h, b);
+                      c * 64, qstart + mblock * 256 + t * 128, h, bc);
       bool ok = true;
       for (int j = JLO; j < JHI && ok; ++j) {
         const int idx = j - JLO, s = idx % S, u = idx / S;
@@ -228,9 +247,9 @@ __global__ void __launch_bounds__(352, 1)
         mbar_arrive_expect_tx(bar_kvfull(s), 2 * Cfg::kTileBytes);
         for (int c = 0; c < D / 64; ++c) {
           tma_load_4d(sbase + Cfg::kSmemK + s * Cfg::kTileBytes + c * Cfg::kChunk, &tmK,
-                      bar_kvfull(s), c * 64, j * 128, g, b);
+                      bar_kvfull(s), c * 64, kstart + j * 128, g, bc);
           tma_load_4d(sbase + Cfg::kSmemV + s * Cfg::kTileBytes + c * Cfg::kChunk, &tmV,
-                      bar_kvfull(s), c * 64, j * 128, g, b);
+                      bar_kvfull(s), c * 64, kstart + j * 128, g, bc);
         }
       }
     }
@@ -415,7 +434,7 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t tP = kSepP ? tmem + lane_base + Cfg::kColP + t * 64 : tS;
     const uint32_t tO = tmem + lane_base + Cfg::kColO + t * D;
     int lo_i, hi_i;
-    row_key_range(row, p.Nq, p.Nk, p.causal, p.wl, p.wr, lo_i, hi_i);
+    row_key_range(row, Nq, Nk, p.causal, p.wl, p.wr, lo_i, hi_i);
     const float sc = p.scale_log2;
     float m_use = -INFINITY;  // running max in scaled log2 units (reference for O and l)
     float l = 0.f;
@@ -536,8 +555,8 @@ __global__ void __launch_bounds__(352, 1)
       const bool has = (n > 0) && (l > 0.f);
       const float inv_l = has ? 1.f / l : 0.f;
       const float lse = has ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const bool store = row < p.Nq;
-      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + b * p.o_sb + int64_t(row) * p.o_ss +
+      const bool store = row < Nq;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + bc * p.o_sb + int64_t(qstart + row) * p.o_ss +
                        int64_t(h) * p.o_sh;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -561,7 +580,12 @@ __global__ void __launch_bounds__(352, 1)
             dst[q4] = make_uint4(pkd[4 * q4], pkd[4 * q4 + 1], pkd[4 * q4 + 2], pkd[4 * q4 + 3]);
         }
       }
-      if (store) p.lse[(int64_t(b) * p.Hq + h) * p.Nq + row] = lse;
+      if (store) {
+        if (p.cu_q != nullptr)
+          p.lse[int64_t(h) * p.total_q + qstart + row] = lse;
+        else
+          p.lse[(int64_t(b) * p.Hq + h) * p.Nq + row] = lse;
+      }
     }
   }
 

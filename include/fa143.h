@@ -90,6 +90,36 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int window_right, void* stream);
 
 /*
+ * Forward pass over a variable-length packed batch (no padding): sequence b
+ * owns query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) of q and o and key rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]) of k and v.  The pages name native
+ * dynamic sequence lengths without padding inputs to a fixed length
+ * ("FlashAttention V3原理与训练推理加速实战指南", section "一、FlashAttention V3
+ * 核心原理革新") and variable sequence lengths among the backend features
+ * ("Что такое FlashAttention…", section "Версии, оборудование и
+ * первоисточники").
+ *   q, o       [total_q, Hq, d]    strides {token, head} in elements
+ *   k, v       [total_k, Hkv, d]   strides {token, head}
+ *   lse        [Hq, total_q] fp32  contiguous, written
+ *   cu_seqlens_q, cu_seqlens_k: device int32 [B + 1], non-decreasing,
+ *              starting at 0 and ending at total_q / total_k
+ *   max_seqlen_q / max_seqlen_k: bounds on the sequence lengths (they size the
+ *              grid).  Masks (causal, window) apply within each sequence, with
+ *              the same bottom-right alignment as fa_fwd.
+ * The offsets are read on the device: lengths are clamped to the max_seqlen
+ * bounds and rows to the totals, so malformed offsets give wrong results but
+ * never an access outside the tensors.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                  int Hq, int Hkv, int d,
+                  const int64_t q_stride[2], const int64_t k_stride[2],
+                  const int64_t v_stride[2], const int64_t o_stride[2],
+                  int dtype, float softmax_scale, int causal, int window_left,
+                  int window_right, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
  * accumulator [B, Nq, Hq, d] and the fp32 row terms D and LSE*log2(e)
  * [B, Hq, Nq].  The caller allocates it (256-byte aligned); its contents
@@ -157,6 +187,25 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                    const int64_t dk_stride[3], const int64_t dv_stride[3],
                    int dtype, float softmax_scale, int causal, int window_left,
                    int window_right, void* stream);
+
+/*
+ * Backward pass over a variable-length packed batch (layouts and offsets as in
+ * fa_fwd_varlen; dq like q, dk and dv like k; lse [Hq, total_q] from
+ * fa_fwd_varlen).  workspace >= fa_bwd_workspace_size(B, max_seqlen_q, Hq, d)
+ * bytes.  Same gradient, accumulation and error behaviour as fa_bwd.
+ */
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                  const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                  void* workspace, size_t workspace_bytes,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                  int Hq, int Hkv, int d,
+                  const int64_t q_stride[2], const int64_t k_stride[2],
+                  const int64_t v_stride[2], const int64_t o_stride[2],
+                  const int64_t do_stride[2], const int64_t dq_stride[2],
+                  const int64_t dk_stride[2], const int64_t dv_stride[2],
+                  int dtype, float softmax_scale, int causal, int window_left,
+                  int window_right, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device error word of

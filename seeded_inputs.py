@@ -94,6 +94,61 @@ def make_workload_inputs(w: Workload, with_dout=None):
                     w.seed, with_dout=with_dout)
 
 
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """A packed batch of independent sequences of mixed length (no padding)."""
+    name: str
+    n_seqs: int
+    min_len: int
+    max_len: int
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    dtype: torch.dtype
+    causal: bool
+    seed: int
+
+    @property
+    def softmax_scale(self) -> float:
+        return float(self.head_dim) ** -0.5
+
+    def lengths(self):
+        g = torch.Generator(device="cpu")
+        g.manual_seed(int(self.seed))
+        return [int(x) for x in torch.randint(self.min_len, self.max_len + 1, (self.n_seqs,),
+                                              generator=g)]
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "sequences": self.n_seqs,
+                "lengths": "uniform in [%d, %d]" % (self.min_len, self.max_len),
+                "q_heads": self.q_heads, "kv_heads": self.kv_heads, "head_dim": self.head_dim,
+                "dtype": str(self.dtype).replace("torch.", ""), "causal": self.causal,
+                "seed": self.seed}
+
+
+VARLEN_WORKLOADS = {
+    "varlen_8seq_512to4096_h16_d128_bf16_causal": VarlenWorkload(
+        "varlen_8seq_512to4096_h16_d128_bf16_causal", 8, 512, 4096, 16, 16, 128, BF16, True,
+        seed=5),
+}
+
+
+def make_varlen_inputs(w: VarlenWorkload):
+    """Packed Q [total, Hq, d], K, V [total, Hkv, d], dO and int32 offsets [B+1]
+    (CPU tensors); drawn in the order Q, K, V, dO after the lengths."""
+    lens = w.lengths()
+    total = sum(lens)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed) + 1)
+    q = torch.randn((total, w.q_heads, w.head_dim), generator=g).to(w.dtype)
+    k = torch.randn((total, w.kv_heads, w.head_dim), generator=g).to(w.dtype)
+    v = torch.randn((total, w.kv_heads, w.head_dim), generator=g).to(w.dtype)
+    do = torch.randn((total, w.q_heads, w.head_dim), generator=g).to(w.dtype)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0).to(torch.int32)
+    return q, k, v, do, cu, lens
+
+
 def sample_rows(batch, q_heads, seqlen_q, n, seed):
     """n distinct (b, h, i) triples, always including the first and last row of
     the sequence so the ragged tail and the causal corner are covered."""

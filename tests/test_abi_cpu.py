@@ -95,3 +95,14 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 8, 1, 64, dtype=torch.float16)
     with pytest.raises(RuntimeError):
         fa.fa_fwd(q, q, q)
+
+
+def test_varlen_rejects_bad_offsets_arguments(lib):
+    st = (ctypes.c_int64 * 2)(256, 64)
+    args = lambda cu_q, cu_k, B, mq, mk, tq, tk: lib.fa_fwd_varlen(  # noqa: E731
+        0x10000, 0x20000, 0x30000, 0x40000, 0x50000, cu_q, cu_k, B, mq, mk, tq, tk, 4, 4, 64,
+        st, st, st, st, 0, 0.125, 1, -1, -1, None)
+    assert args(0, 0x60000, 2, 10, 10, 20, 20) == fa.FA_ERR_INVALID_ARG      # no offsets
+    assert args(0x60002, 0x60000, 2, 10, 10, 20, 20) == fa.FA_ERR_ALIGNMENT  # misaligned
+    assert args(0x60000, 0x60000, 2, 30, 10, 20, 20) == fa.FA_ERR_INVALID_ARG  # max > total
+    assert args(0x60000, 0x60000, 0, 10, 10, 20, 20) == fa.FA_ERR_INVALID_ARG  # no sequences
