@@ -30,12 +30,13 @@
 //      TMA bulk reduce-adds staged through shared memory.
 //   3. fa_bwd_dq_convert_kernel: dQ accumulator -> dQ in the input dtype.
 //
-// Roles (480 threads): warps 0-7 compute (thread = key row = tensor-memory
+// Roles (512 threads): warps 0-7 compute (thread = key row = tensor-memory
 // lane; warps 0-3 take queries 0-63 of a tile, warps 4-7 queries 64-127),
 // warps 8-11 move dQ out of tensor memory into a staging buffer, warp 14
 // reduces the staged rows into the fp32 accumulator (TMA bulk reduce-add),
 // warp 12 issues the MMAs (one elected lane of a converged warp), warp 13
-// issues TMA loads.  dO has one buffer, refilled as soon as dV has read it;
+// issues TMA loads, warp 15 idles (it completes warpgroup 3, whose registers
+// go to the dQ warpgroup).  dO has one buffer, refilled as soon as dV has read it;
 // that frees the staging buffer so the compute warps never wait for dQ.
 // Tensor memory: two 128-column regions R0/R1 swap roles every step (S, P, dQ
 // in one; dP, dS in the other), dK at 256, dV at 256 + d.  Per step the MMA
@@ -192,7 +193,13 @@ template <int D>
 struct BwdCfg {
   static constexpr int kChunk = 128 * 64 * 2;     // 128 rows x 64 columns, 16-bit, swizzled
   static constexpr int kTileBytes = 128 * D * 2;  // a 128-row tile
-  static constexpr int kThreads = 480;
+  static constexpr int kThreads = 512;
+  // registers per thread: launched with 65536 / 512 = 128; warpgroup 3 (MMA,
+  // TMA, reduce issuer, one idle warp) gives some to warpgroup 2 (dQ readout):
+  // 128 * (128 + 128 + kRegsDq + kRegsCtl) must equal 512 * 128
+  static constexpr int kRegsLaunch = 128;
+  static constexpr int kRegsDq = 168;
+  static constexpr int kRegsCtl = 88;
   static constexpr int kSmemK = 0;
   static constexpr int kSmemV = kSmemK + kTileBytes;
   static constexpr int kSmemQ = kSmemV + kTileBytes;        // 2 stages
@@ -221,7 +228,7 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(480, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
@@ -317,8 +324,14 @@ __global__ void __launch_bounds__(480, 1)
   auto wait_all = [&](uint32_t bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
   };
+  static_assert(128 * (2 * Cfg::kRegsLaunch + Cfg::kRegsDq + Cfg::kRegsCtl) ==
+                    Cfg::kThreads * Cfg::kRegsLaunch,
+                "register split must add up to the launch budget");
 
-  if (warp == 13) {
+  if (warp >= 12) {
+   // warpgroup 3 hands registers to the dQ warpgroup (same instruction for all 4 warps)
+   regs_dec<Cfg::kRegsCtl>();
+   if (warp == 13) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && T > 0) {
       tma_prefetch_desc(&tmQ);
@@ -352,7 +365,7 @@ __global__ void __launch_bounds__(480, 1)
                       qstart + m * 128, h, bc);
       }
     }
-  } else if (warp == 14) {
+   } else if (warp == 14) {
     // ------------------------------------------------------------ dQ reduce issuer
     // Once a round of dQ rows is staged, one elected lane reduces it into the
     // fp32 accumulator (two bulk tensor reduce-adds of 32 columns x 128 rows)
@@ -378,7 +391,7 @@ __global__ void __launch_bounds__(480, 1)
       if (elect_one()) bulk_wait0();  // reduce-adds complete before the CTA exits
       __syncwarp();
     }
-  } else if (warp == 12) {
+   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop and waits; one elected lane issues each
     // batch of MMAs and its commits.
@@ -389,14 +402,21 @@ __global__ void __launch_bounds__(480, 1)
       // descriptors are built once; an MMA only adds a compile-time offset
       constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
       constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // MN-major tiles
-      const uint64_t dK_k = sdesc_at(kDescK, sbase + Cfg::kSmemK);
-      const uint64_t dV_k = sdesc_at(kDescK, sbase + Cfg::kSmemV);
-      const uint64_t dK_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemK);
-      const uint64_t dDS_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDS);
-      const uint64_t dQ_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
-      const uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
-      const uint64_t dDO_k = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
-      const uint64_t dDO_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
+      uint64_t dK_k = sdesc_at(kDescK, sbase + Cfg::kSmemK);
+      uint64_t dV_k = sdesc_at(kDescK, sbase + Cfg::kSmemV);
+      uint64_t dK_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemK);
+      uint64_t dDS_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDS);
+      uint64_t dQ_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
+      uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
+      uint64_t dDO_k = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
+      uint64_t dDO_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
+      // This warp runs on a reduced register budget: hide the bases from the
+      // optimiser once per step so it adds the offsets where they are used
+      // instead of keeping every base + offset live across the loop.
+      auto opaque_bases = [&]() {
+        asm volatile("" : "+l"(dK_k), "+l"(dV_k), "+l"(dK_mn), "+l"(dDS_mn));
+        asm volatile("" : "+l"(dQ_k0), "+l"(dQ_mn0), "+l"(dDO_k), "+l"(dDO_mn));
+      };
       // S^T(s) = K Q_s^T into region r (M = keys, N = queries, K-dim = d)
       auto issue_s = [&](int s, uint32_t r) {
         const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
@@ -437,6 +457,7 @@ __global__ void __launch_bounds__(480, 1)
         }
       }
       for (int s = 0; s < T && ok; ++s) {
+        opaque_bases();
         const int st = s & 1;
         const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
         const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
@@ -487,7 +508,9 @@ __global__ void __launch_bounds__(480, 1)
         }
       }
     }
+   }  // warp 15 idles
   } else if (warp >= 8) {
+    regs_inc<Cfg::kRegsDq>();
     // ------------------------------------------------------------ dQ readout (warps 8-11)
     // dQ(s) leaves tensor memory (thread = query row r) 64 columns at a time;
     // scale * dQ is staged, 128-byte swizzled, in the staging buffer for the
@@ -502,24 +525,27 @@ __global__ void __launch_bounds__(480, 1)
       if (!(ok = wait_all(bar_dq, s & 1))) break;
       tc_fence_after();
       const uint32_t R = tmem + lane_base + (s & 1) * 128;
-      for (int rd = 0; rd < kR && ok; ++rd) {
-        uint32_t v[64];
-        tmem_ld32(R + rd * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(R + rd * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        if (rd == kR - 1) {  // dQ(s) is out of tensor memory: the region may be reused
-          tc_fence_before();
-          mbar_arrive(bar_dqfree);
-        }
+      // all of dQ(s) into registers, then the region is released at once
+      uint32_t v[D];
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32)
+        tmem_ld32(R + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_dqfree);
+#pragma unroll
+      for (int rd = 0; rd < kR; ++rd) {
         // the previous round's staging must have been read by the TMA unit
+        // (no early exit here: the loop must unroll so v stays in registers)
         const int prev = s * kR + rd - 1;
-        if (prev >= 0 && !(ok = wait_all(bar_roundfree, prev & 1))) break;
+        if (ok && prev >= 0) ok = wait_all(bar_roundfree, prev & 1);
+        if (!ok) continue;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint8_t* chunk = stage + c * (128 * 128) + r * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float* x = reinterpret_cast<const float*>(&v[c * 32 + u * 4]);
+            const float* x = reinterpret_cast<const float*>(&v[rd * 64 + c * 32 + u * 4]);
             *reinterpret_cast<float4*>(chunk + ((u ^ (r & 7)) * 16)) =
                 make_float4(x[0] * p.scale, x[1] * p.scale, x[2] * p.scale, x[3] * p.scale);
           }
