@@ -26,22 +26,25 @@
 //                                                    smem as the dQ operand)
 //        dK  += dS^T Q_i       (A = dS^T from tensor memory)
 //        dQ_i = dS K           (A = dS from smem, MN-major)
-//      and the compute warps add scale * dQ_i into the fp32 accumulator with
-//      TMA bulk reduce-adds staged through shared memory.
+//      and scale * dQ_i is added into the fp32 accumulator with TMA bulk
+//      reduce-adds staged through shared memory.
 //   3. fa_bwd_dq_convert_kernel: dQ accumulator -> dQ in the input dtype.
 //
 // Roles (512 threads): warps 0-7 compute (thread = key row = tensor-memory
 // lane; warps 0-3 take queries 0-63 of a tile, warps 4-7 queries 64-127),
 // warps 8-11 move dQ out of tensor memory into a staging buffer, warp 14
 // reduces the staged rows into the fp32 accumulator (TMA bulk reduce-add),
-// warp 12 issues the MMAs (one elected lane of a converged warp), warp 13
-// issues TMA loads, warp 15 idles (it completes warpgroup 3, whose registers
-// go to the dQ warpgroup).  dO has one buffer, refilled as soon as dV has read it;
-// that frees the staging buffer so the compute warps never wait for dQ.
-// Tensor memory: two 128-column regions R0/R1 swap roles every step (S, P, dQ
-// in one; dP, dS in the other), dK at 256, dV at 256 + d.  Per step the MMA
-// order is dV(s), dK(s), S(s+1), dQ(s), dP(s+1); dQ(s) is reduced while the
-// compute warps work on step s+1.
+// warp 13 issues TMA loads, and two warps issue MMAs (one elected lane of a
+// converged warp each): warp 15 the S^T and dP^T products the compute warps
+// wait for, warp 12 the dV, dK and dQ accumulations.  Warpgroup 3 (warps
+// 12-15) runs on fewer registers so the dQ warpgroup can hold a whole dQ row.
+// dO has one buffer, refilled as soon as dP^T and dV have read it; that frees
+// the staging buffer so the compute warps never wait for dQ.
+// Tensor memory: two 128-column regions R0/R1 swap roles every step.  The
+// region of step s holds S^T(s), then P^T(s) and dS^T(s) packed side by side,
+// then dQ(s), then dP^T(s+1); the other holds dP^T(s), then S^T(s+1).  dK sits
+// at column 256, dV at 256 + d.  S^T(s+1) is computed as soon as the compute
+// warps have read dP^T(s), during the dS phase of step s.
 #pragma once
 
 #include <climits>
@@ -198,8 +201,8 @@ struct BwdCfg {
   // TMA, reduce issuer, one idle warp) gives some to warpgroup 2 (dQ readout):
   // 128 * (128 + 128 + kRegsDq + kRegsCtl) must equal 512 * 128
   static constexpr int kRegsLaunch = 128;
-  static constexpr int kRegsDq = 168;
-  static constexpr int kRegsCtl = 88;
+  static constexpr int kRegsDq = 160;
+  static constexpr int kRegsCtl = 96;
   static constexpr int kSmemK = 0;
   static constexpr int kSmemV = kSmemK + kTileBytes;
   static constexpr int kSmemQ = kSmemV + kTileBytes;        // 2 stages
@@ -255,6 +258,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t bar_dqfree = smem_u32(&bars[12]);
   const uint32_t bar_staged = smem_u32(&bars[13]);     // a dQ round staged (128 arrivals)
   const uint32_t bar_roundfree = smem_u32(&bars[14]);  // staged round read by the TMA unit
+  const uint32_t bar_dpfree = smem_u32(&bars[15]);     // dP^T read out of tensor memory (256)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kSmemBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kSmemBar + 200);
 
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_qempty(st), 1);
     }
     mbar_init(bar_dofull, 1);
-    mbar_init(bar_doempty, 1);
+    mbar_init(bar_doempty, 2);  // one commit from each MMA issuer
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
     mbar_init(bar_p, 256);
@@ -305,6 +309,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(bar_dqfree, 128);
     mbar_init(bar_staged, 128);
     mbar_init(bar_roundfree, 1);
+    mbar_init(bar_dpfree, 256);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -391,124 +396,137 @@ __global__ void __launch_bounds__(512, 1)
       if (elect_one()) bulk_wait0();  // reduce-adds complete before the CTA exits
       __syncwarp();
     }
-   } else if (warp == 12) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs this loop and waits; one elected lane issues each
-    // batch of MMAs and its commits.
+   } else {
+    // ------------------------------------------------------------ MMA issuers
+    // Two warps issue MMAs, each running its whole loop and waiting as a
+    // converged warp while one elected lane issues a batch and its commits:
+    //   warp 15: S^T(s) and dP^T(s), the products the compute warps wait for;
+    //   warp 12: dV(s), dK(s), dQ(s), the accumulations.
+    // A commit tracks only the committing thread's MMAs; dO is read by both
+    // warps, so its buffer is released by one commit from each.
     if (T > 0) {
       const uint32_t idesc_ss = make_idesc_f16(BF16, 128, 128, false, false);   // S^T, dP^T
       const uint32_t idesc_acc = make_idesc_f16(BF16, 128, D, false, true);    // dV, dK
       const uint32_t idesc_dq = make_idesc_f16(BF16, 128, D, true, true);      // dQ
-      // descriptors are built once; an MMA only adds a compile-time offset
       constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
       constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // MN-major tiles
-      uint64_t dK_k = sdesc_at(kDescK, sbase + Cfg::kSmemK);
-      uint64_t dV_k = sdesc_at(kDescK, sbase + Cfg::kSmemV);
-      uint64_t dK_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemK);
-      uint64_t dDS_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDS);
-      uint64_t dQ_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
-      uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
-      uint64_t dDO_k = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
-      uint64_t dDO_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
-      // This warp runs on a reduced register budget: hide the bases from the
-      // optimiser once per step so it adds the offsets where they are used
-      // instead of keeping every base + offset live across the loop.
-      auto opaque_bases = [&]() {
-        asm volatile("" : "+l"(dK_k), "+l"(dV_k), "+l"(dK_mn), "+l"(dDS_mn));
-        asm volatile("" : "+l"(dQ_k0), "+l"(dQ_mn0), "+l"(dDO_k), "+l"(dDO_mn));
-      };
-      // S^T(s) = K Q_s^T into region r (M = keys, N = queries, K-dim = d)
-      auto issue_s = [&](int s, uint32_t r) {
-        const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(r, dK_k + o, dQ_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_s);
-        }
-        __syncwarp();
-      };
-      // dP^T(s) = V dO_s^T into region r
-      auto issue_dp = [&](uint32_t r) {
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(r, dV_k + o, dDO_k + o, idesc_ss, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_dp);
-        }
-        __syncwarp();
-      };
-      // P^T and dS^T sit in columns [0, 32) (queries 0-63) and [64, 96)
-      // (queries 64-127) of their region: 16 queries per K step = 8 columns
-      auto acol = [](int kk) { return uint32_t(kk < 4 ? kk * 8 : 64 + (kk - 4) * 8); };
       bool ok = wait_all(bar_kv, 0);
-      if (ok) ok = wait_all(bar_qfull(0), 0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, tmem);
-        ok = wait_all(bar_dofull, 0);
+      if (warp == 15) {
+        uint64_t dK_k = sdesc_at(kDescK, sbase + Cfg::kSmemK);
+        uint64_t dV_k = sdesc_at(kDescK, sbase + Cfg::kSmemV);
+        uint64_t dQ_k0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
+        uint64_t dDO_k = sdesc_at(kDescK, sbase + Cfg::kSmemDO);
+        // on a reduced register budget: hide the bases from the optimiser once
+        // per step so base + offset is formed where it is used
+        auto opaque_bases = [&]() {
+          asm volatile("" : "+l"(dK_k), "+l"(dV_k), "+l"(dQ_k0), "+l"(dDO_k));
+        };
+        // S^T(s) = K Q_s^T into region r (M = keys, N = queries, K-dim = d)
+        auto issue_s = [&](int s, uint32_t r) {
+          const uint64_t stoff = uint64_t(((s & 1) * Cfg::kTileBytes) >> 4);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+              mma_ss(r, dK_k + o, dQ_k0 + stoff + o, idesc_ss, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_s);
+          }
+          __syncwarp();
+        };
+        // dP^T(s) = V dO_s^T into region r; dO is then free as far as this warp goes
+        auto issue_dp = [&](uint32_t r) {
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t o = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
+              mma_ss(r, dV_k + o, dDO_k + o, idesc_ss, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_dp);
+            mma_commit(bar_doempty);
+          }
+          __syncwarp();
+        };
+        if (ok) ok = wait_all(bar_qfull(0), 0);
         if (ok) {
           tc_fence_after();
-          issue_dp(tmem + 128);
+          issue_s(0, tmem);
+          ok = wait_all(bar_dofull, 0);
+          if (ok) {
+            tc_fence_after();
+            issue_dp(tmem + 128);
+          }
         }
-      }
-      for (int s = 0; s < T && ok; ++s) {
-        opaque_bases();
-        const int st = s & 1;
-        const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
-        const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
-        const uint32_t acc0 = s > 0 ? 1u : 0u;
-        // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major); dO is then free
-        if (!(ok = wait_all(bar_p, s & 1))) break;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Cfg::kColDV, Ra + acol(kk), dDO_mn + uint64_t((kk * 2048) >> 4),
-                   idesc_acc, kk > 0 ? 1u : acc0);
-          mma_commit(bar_doempty);
-        }
-        __syncwarp();
-        // dK += dS^T Q (A = dS^T from tensor memory, B = Q MN-major)
-        if (!(ok = wait_all(bar_ds, s & 1))) break;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Cfg::kColDK, Rb + acol(kk),
-                   dQ_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
-          mma_commit(bar_qempty(st));  // Q_s, LSE_s, D_s are no longer read
-        }
-        __syncwarp();
-        // S^T(s+1) into Rb (its dS^T has just been consumed by dK)
-        if (s + 1 < T) {
+        for (int s = 0; s + 1 < T && ok; ++s) {
+          opaque_bases();
+          const uint32_t Ra = tmem + (s & 1) * 128, Rb = tmem + ((s + 1) & 1) * 128;
+          // S^T(s+1) into Rb once the compute warps hold dP^T(s) in registers
+          if (!(ok = wait_all(bar_dpfree, s & 1))) break;
           if (!(ok = wait_all(bar_qfull((s + 1) & 1), ((s + 1) >> 1) & 1))) break;
           tc_fence_after();
           issue_s(s + 1, Rb);
-        }
-        // dQ(s) = dS K into Ra (A = dS from smem, MN-major; B = K MN-major)
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(Ra, dDS_mn + uint64_t((kk * 2048) >> 4), dK_mn + uint64_t((kk * 2048) >> 4),
-                   idesc_dq, kk > 0 ? 1u : 0u);
-          mma_commit(bar_dq);
-        }
-        __syncwarp();
-        // dP^T(s+1) into Ra once dQ(s) has been read out of it and dO(s+1) is in
-        if (s + 1 < T) {
-          if (!(ok = wait_all(bar_dqfree, s & 1))) break;
+          // dP^T(s+1) into Ra once dO(s+1) is in (normally long since) and dQ(s)
+          // has been read out of Ra (the wait on the critical path comes last)
           if (!(ok = wait_all(bar_dofull, (s + 1) & 1))) break;
+          if (!(ok = wait_all(bar_dqfree, s & 1))) break;
           tc_fence_after();
           issue_dp(Ra);
         }
+      } else if (warp == 12) {
+        uint64_t dK_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemK);
+        uint64_t dDS_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDS);
+        uint64_t dQ_mn0 = sdesc_at(kDescMN, sbase + Cfg::kSmemQ);
+        uint64_t dDO_mn = sdesc_at(kDescMN, sbase + Cfg::kSmemDO);
+        auto opaque_bases = [&]() {
+          asm volatile("" : "+l"(dK_mn), "+l"(dDS_mn), "+l"(dQ_mn0), "+l"(dDO_mn));
+        };
+        // P^T sits in columns [0, 32) (queries 0-63) and [64, 96) (queries
+        // 64-127) of its region, dS^T 32 columns further: 16 queries per K
+        // step = 8 columns
+        auto acol = [](int kk) { return uint32_t(kk < 4 ? kk * 8 : 64 + (kk - 4) * 8); };
+        for (int s = 0; s < T && ok; ++s) {
+          opaque_bases();
+          const int st = s & 1;
+          const uint32_t Ra = tmem + (s & 1) * 128;
+          const uint64_t stoff = uint64_t((st * Cfg::kTileBytes) >> 4);
+          const uint32_t acc0 = s > 0 ? 1u : 0u;
+          // dV += P^T dO (A = P^T from tensor memory, B = dO MN-major)
+          if (!(ok = wait_all(bar_dofull, s & 1))) break;
+          if (!(ok = wait_all(bar_p, s & 1))) break;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + Cfg::kColDV, Ra + acol(kk), dDO_mn + uint64_t((kk * 2048) >> 4),
+                     idesc_acc, kk > 0 ? 1u : acc0);
+            mma_commit(bar_doempty);
+          }
+          __syncwarp();
+          // dK += dS^T Q (A = dS^T from tensor memory, beside P^T; B = Q MN-major)
+          if (!(ok = wait_all(bar_qfull(st), (s >> 1) & 1))) break;
+          if (!(ok = wait_all(bar_ds, s & 1))) break;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + Cfg::kColDK, Ra + 32 + acol(kk),
+                     dQ_mn0 + stoff + uint64_t((kk * 2048) >> 4), idesc_acc, kk > 0 ? 1u : acc0);
+            mma_commit(bar_qempty(st));  // Q_s, LSE_s, D_s are no longer read
+          }
+          __syncwarp();
+          // dQ(s) = dS K into Ra (A = dS from smem, MN-major; B = K MN-major)
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(Ra, dDS_mn + uint64_t((kk * 2048) >> 4), dK_mn + uint64_t((kk * 2048) >> 4),
+                     idesc_dq, kk > 0 ? 1u : 0u);
+            mma_commit(bar_dq);
+          }
+          __syncwarp();
+        }
       }
     }
-   }  // warp 15 idles
+   }
   } else if (warp >= 8) {
     regs_inc<Cfg::kRegsDq>();
     // ------------------------------------------------------------ dQ readout (warps 8-11)
@@ -625,48 +643,55 @@ __global__ void __launch_bounds__(512, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
-      // dS^T = P^T * (dP^T - D), to tensor memory and to smem (dQ operand);
-      // the dQ(s-1) MMA, the last reader of the smem buffer, completed before
-      // dP^T(s) was issued
+      // dS^T = P^T * (dP^T - D), to tensor memory (beside P^T) and to smem (dQ
+      // operand); the dQ(s-1) MMA, the last reader of the smem buffer,
+      // completed before dP^T(s) was issued.  dP^T(s) is read out first so
+      // that S^T(s+1) can be computed into its region during this phase.
       if (!(ok = wait_all(bar_dp, s & 1))) break;
       tc_fence_after();
       uint8_t* dsrow = smem + Cfg::kSmemDS + half * Cfg::kChunk + j * 128;
+      uint32_t dpr[64];
+      tmem_ld32(Rb + colS, *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]));
+      tmem_ld32(Rb + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_dpfree);
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t dpr[32], pr[16];
-        tmem_ld32(Rb + colS + c0, dpr);
+        uint32_t pr[16], dk[16];
         tmem_ld16(Ra + colP + c0 / 2, pr);
         tmem_wait_ld();
-        uint32_t dk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const float4 d4 = *reinterpret_cast<const float4*>(Dv + c0 + c);
+          const uint32_t pa = pr[c / 2], pb = pr[c / 2 + 1];
           float pf[4];
           if constexpr (BF16) {
-            pf[0] = __uint_as_float(pr[c / 2] << 16);
-            pf[1] = __uint_as_float(pr[c / 2] & 0xFFFF0000u);
-            pf[2] = __uint_as_float(pr[c / 2 + 1] << 16);
-            pf[3] = __uint_as_float(pr[c / 2 + 1] & 0xFFFF0000u);
+            pf[0] = __uint_as_float(pa << 16);
+            pf[1] = __uint_as_float(pa & 0xFFFF0000u);
+            pf[2] = __uint_as_float(pb << 16);
+            pf[3] = __uint_as_float(pb & 0xFFFF0000u);
           } else {
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&pr[c / 2]));
-            const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&pr[c / 2 + 1]));
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&pa));
+            const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&pb));
             pf[0] = a.x;
             pf[1] = a.y;
             pf[2] = bb.x;
             pf[3] = bb.y;
           }
           const float2 d01 = __fmul2_rn(make_float2(pf[0], pf[1]),
-                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c]),
-                                                               __uint_as_float(dpr[c + 1])),
+                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c0 + c]),
+                                                               __uint_as_float(dpr[c0 + c + 1])),
                                                    make_float2(-d4.x, -d4.y)));
           const float2 d23 = __fmul2_rn(make_float2(pf[2], pf[3]),
-                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c + 2]),
-                                                               __uint_as_float(dpr[c + 3])),
+                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c0 + c + 2]),
+                                                               __uint_as_float(dpr[c0 + c + 3])),
                                                    make_float2(-d4.z, -d4.w)));
           dk[c / 2] = pack2<BF16>(d01.x, d01.y);
           dk[c / 2 + 1] = pack2<BF16>(d23.x, d23.y);
         }
-        tmem_st16(Rb + colP + c0 / 2, dk);
+        // columns of S^T(s) this thread has already read
+        tmem_st16(Ra + colP + 32 + c0 / 2, dk);
         // smem copy in the MN-major 128-byte-swizzled layout of the dQ A operand:
         // chunk `half` holds queries [64 half, 64 half + 64) of every key row;
         // the 16-byte unit u of row j sits at unit u ^ (j % 8).
