@@ -76,9 +76,16 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# the sources each profiled kernel is compiled from (device code only)
+KERNEL_SOURCES = {
+    "fa_bwd_main_kernel": ("fa_bwd.cuh", "fa_exp2.cuh", "fa_ptx.cuh"),
+    "fa_fwd_kernel": ("fa_fwd.cuh", "fa_exp2.cuh", "fa_ptx.cuh"),
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for name in ("fa_bwd.cuh", "fa_fwd.cuh", "fa_ptx.cuh", "fa143_api.cu"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "exact_attention_143_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -94,7 +101,7 @@ def load_traffic(kernel):
     except (OSError, ValueError):
         return None
     ent = tr.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -52,7 +52,7 @@
 #include <cuda_fp16.h>
 
 #include "fa_ptx.cuh"
-#include "fa_fwd.cuh"  // exp2_fma_pair
+#include "fa_exp2.cuh"
 
 namespace fa {
 
