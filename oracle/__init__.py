@@ -81,6 +81,9 @@ class Oracle:
         lib.oracle_probs.restype = i
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp] + shape + [i]
         lib.oracle_bwd.restype = i
+        ipt = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_fwd_paged.argtypes = [dp, dp, dp, ipt, ipt, dp, dp] + [i] * 8 + [dbl, i, i, i, i]
+        lib.oracle_fwd_paged.restype = i
         lib.oracle_default_threads.argtypes = []
         lib.oracle_default_threads.restype = i
         self.lib = lib
@@ -133,6 +136,36 @@ class Oracle:
             raise RuntimeError("oracle_probs failed")
         return p
 
+    def attention_fwd_paged(self, q, k_cache, v_cache, block_table, cache_seqlens, softmax_scale,
+                            causal=False, window_size=(-1, -1), nthreads=0):
+        """O [B,Nq,Hq,d] and LSE [B,Hq,Nq] of q against a paged KV cache.
+
+        ``k_cache``/``v_cache`` are [num_pages, page_size, Hkv, d];
+        ``block_table`` is int [B, max_pages_per_seq]; sequence b holds
+        ``cache_seqlens[b]`` keys."""
+        q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+        if q.ndim != 4 or kc.ndim != 4 or vc.shape != kc.shape:
+            raise ValueError("q must be [B,Nq,Hq,d] and the caches [pages,page_size,Hkv,d]")
+        B, Nq, Hq, d = q.shape
+        num_pages, P, Hkv, dk = kc.shape
+        if dk != d or Hq % Hkv:
+            raise ValueError("inconsistent q / cache shapes")
+        bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+        sl = np.ascontiguousarray(np.asarray(cache_seqlens, dtype=np.int32))
+        if bt.ndim != 2 or bt.shape[0] != B or sl.shape != (B,):
+            raise ValueError("block_table must be [B, max_pages] and cache_seqlens [B]")
+        o = np.zeros((B, Nq, Hq, d), np.float64)
+        lse = np.zeros((B, Hq, Nq), np.float64)
+        c, wl, wr = _mask_args(causal, window_size)
+        ipt = ctypes.POINTER(ctypes.c_int)
+        rc = self.lib.oracle_fwd_paged(_ptr(q), _ptr(kc), _ptr(vc), bt.ctypes.data_as(ipt),
+                                       sl.ctypes.data_as(ipt), _ptr(o), _ptr(lse), B, Nq, Hq,
+                                       Hkv, d, P, num_pages, bt.shape[1], float(softmax_scale),
+                                       c, wl, wr, int(nthreads))
+        if rc:
+            raise RuntimeError("oracle_fwd_paged failed (bad seqlen or page id?)")
+        return o, lse
+
     def attention_bwd(self, q, k, v, dout, softmax_scale, causal=False, window_size=(-1, -1),
                       nthreads=0):
         """dQ, dK, dV of L = sum(dout * O), plus the oracle's own LSE and D (fp64)."""
@@ -180,3 +213,7 @@ def attention_probs(*a, **kw):
 
 def attention_bwd(*a, **kw):
     return _get().attention_bwd(*a, **kw)
+
+
+def attention_fwd_paged(*a, **kw):
+    return _get().attention_fwd_paged(*a, **kw)

@@ -213,6 +213,85 @@ int oracle_fwd(const double* q, const double* k, const double* v, double* o, dou
     return run_pool(fwd_item, &c, (long)B * Hq * Nq, 2 * (size_t)Nk, nthreads);
 }
 
+/* ------------------------------------------------------------------ */
+/* forward over a paged KV cache                                        */
+/* ------------------------------------------------------------------ */
+/* The keys and values of sequence b are the first cache_seqlens[b] rows of
+ * a cache made of fixed-size pages ("optimizing-attention-flash", the list of
+ * advanced features, which names a paged KV cache; "FlashAttention V3
+ * 原理与…实战指南", section 四 on inference, where the KV cache is kept in
+ * pages and the vLLM example sets a page of 16 tokens): logical key j of
+ * sequence b is row j % P of page block_table[b][j / P], and a page is laid
+ * out [P, Hkv, d].  With the keys gathered that way the result is the
+ * definition above, the mask aligned bottom-right against cache_seqlens[b]
+ * (decode: the Nq new queries are the last Nq positions of the sequence). */
+typedef struct {
+    int B, Nq, Hq, Hkv, d, P, max_pages;
+    double tau;
+    int causal, wl, wr;
+    const double *q, *kc, *vc;
+    const int *block_table, *seqlens;
+    double *o, *lse;
+} paged_ctx;
+
+/* Row of the cache holding logical key j of sequence b, kv head g. */
+static const double* paged_key(const paged_ctx* c, const double* cache, int b, long j, int g) {
+    long page = c->block_table[(size_t)b * c->max_pages + j / c->P];
+    long row = j % c->P;
+    return cache + (((size_t)page * c->P + row) * c->Hkv + g) * c->d;
+}
+
+static void paged_item(void* ctx, long item, double* scratch) {
+    const paged_ctx* c = (const paged_ctx*)ctx;
+    int i = (int)(item % c->Nq);
+    long bh = item / c->Nq;
+    int h = (int)(bh % c->Hq);
+    int b = (int)(bh / c->Hq);
+    int kv_head = h / (c->Hq / c->Hkv);
+    int nk = c->seqlens[b];
+    /* the sequence's own shape, for the shared mask and LSE definitions */
+    shape_t s = {1, c->Nq, nk, c->Hq, c->Hkv, c->d, c->tau, c->causal, c->wl, c->wr};
+    double* srow = scratch;
+    double* prow = scratch + (nk > 0 ? nk : 1);
+    const double* qi = c->q + (((size_t)b * c->Nq + i) * c->Hq + h) * c->d;
+    for (long j = 0; j < nk; ++j)
+        srow[j] = c->tau * dot(qi, paged_key(c, c->kc, b, j, kv_head), c->d);
+    double l = row_lse(&s, i, srow);
+    prob_row(&s, i, srow, l, prow);
+    double* oi = c->o + (((size_t)b * c->Nq + i) * c->Hq + h) * c->d;
+    for (int cc = 0; cc < c->d; ++cc) oi[cc] = 0.0;
+    for (long j = 0; j < nk; ++j) {
+        if (prow[j] == 0.0) continue;
+        const double* vrow = paged_key(c, c->vc, b, j, kv_head);
+        for (int cc = 0; cc < c->d; ++cc) oi[cc] += prow[j] * vrow[cc];
+    }
+    c->lse[((size_t)b * c->Hq + h) * c->Nq + i] = l;
+}
+
+int oracle_fwd_paged(const double* q, const double* k_cache, const double* v_cache,
+                     const int* block_table, const int* cache_seqlens, double* o, double* lse,
+                     int B, int Nq, int Hq, int Hkv, int d, int page_size, int num_pages,
+                     int max_pages_per_seq, double tau, int causal, int window_left,
+                     int window_right, int nthreads) {
+    if (B < 1 || Nq < 1 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv) return -1;
+    if (page_size < 1 || num_pages < 1 || max_pages_per_seq < 1) return -1;
+    long longest = 0;
+    for (int b = 0; b < B; ++b) {
+        long nk = cache_seqlens[b];
+        if (nk < 0 || nk > (long)max_pages_per_seq * page_size) return -1;
+        for (long pg = 0; pg * page_size < nk; ++pg) {
+            int id = block_table[(size_t)b * max_pages_per_seq + pg];
+            if (id < 0 || id >= num_pages) return -1;
+        }
+        if (nk > longest) longest = nk;
+    }
+    paged_ctx c = {B, Nq, Hq, Hkv, d, page_size, max_pages_per_seq, tau, causal,
+                   window_left, window_right, q, k_cache, v_cache, block_table,
+                   cache_seqlens, o, lse};
+    return run_pool(paged_item, &c, (long)B * Hq * Nq, 2 * (size_t)(longest > 0 ? longest : 1),
+                    nthreads);
+}
+
 static void fwd_rows_item(void* ctx, long item, double* scratch) {
     const fwd_ctx* c = (const fwd_ctx*)ctx;
     int b = (int)c->rows[3 * item], h = (int)c->rows[3 * item + 1], i = (int)c->rows[3 * item + 2];

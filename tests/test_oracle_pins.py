@@ -13,7 +13,10 @@ Each check below ties the oracle to a source independent of its code:
     блоки 2×2"): 16 blocks visited in row-major order, each loaded, attended
     and folded into the output with correct normalisation, must equal full
     attention;
-  * central finite differences and fp64 torch autograd for the backward.
+  * central finite differences and fp64 torch autograd for the backward;
+  * for the paged KV cache, equality with the (pinned) contiguous definition
+    on the gathered keys, through a permuted page table with unrelated
+    values in every row and page the sequence does not own.
 A mutation test then plants plausible mistakes in copies of the oracle's C
 source and checks that these pins catch every one of them.
 """
@@ -345,9 +348,60 @@ def check_empty_rows(orc):
     assert (dq[0, :3] == 0).all()
 
 
+def scatter_to_pages(k, v, P, extra_pages, seed):
+    """Paged caches [pages, P, Hkv, d] holding k/v [B, N, Hkv, d] in a random
+    page order; rows past N and the spare pages hold unrelated values, and
+    every block-table entry (used or not) names a valid page."""
+    B, N, Hkv, d = k.shape
+    per_seq = (N + P - 1) // P
+    n_pages = B * per_seq + extra_pages
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(n_pages)
+    kc = 50.0 * rng.standard_normal((n_pages, P, Hkv, d))
+    vc = 50.0 * rng.standard_normal((n_pages, P, Hkv, d))
+    bt = np.zeros((B, per_seq + 2), np.int32)
+    for b in range(B):
+        for pg in range(per_seq + 2):
+            bt[b, pg] = perm[b * per_seq + pg] if pg < per_seq else perm[(-1 - pg) % n_pages]
+        for j in range(N):
+            kc[bt[b, j // P], j % P] = k[b, j]
+            vc[bt[b, j // P], j % P] = v[b, j]
+    return kc, vc, bt
+
+
+def check_paged(orc):
+    # a paged cache read through its block table equals the contiguous
+    # definition on the gathered keys, for every mask and GQA grouping
+    for (causal, window), (Hq, Hkv), P in itertools.product(MASKS, [(4, 4), (4, 2)], [4, 8]):
+        B, Nq, N, d = 3, 3, 13, 5
+        q, k, v = rand((B, Nq, Hq, d), 121), rand((B, N, Hkv, d), 122), rand((B, N, Hkv, d), 123)
+        kc, vc, bt = scatter_to_pages(k, v, P, 3, 124)
+        o, lse = orc.attention_fwd_paged(q, kc, vc, bt, [N] * B, 0.6, causal, window)
+        oc, lsec = orc.attention_fwd(q, k, v, 0.6, causal, window)
+        np.testing.assert_allclose(o, oc, rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(np.isinf(lse), np.isinf(lsec))
+        fin = np.isfinite(lsec)
+        np.testing.assert_allclose(lse[fin], lsec[fin], rtol=0, atol=1e-12)
+    # ragged lengths: each sequence is its own problem, aligned bottom-right
+    # against its own length; an empty sequence gives O = 0 and LSE = -inf
+    B, Nq, N, Hq, Hkv, d, P = 4, 2, 21, 4, 2, 6, 8
+    q, k, v = rand((B, Nq, Hq, d), 131), rand((B, N, Hkv, d), 132), rand((B, N, Hkv, d), 133)
+    kc, vc, bt = scatter_to_pages(k, v, P, 2, 134)
+    lens = [21, 1, 0, 9]
+    o, lse = orc.attention_fwd_paged(q, kc, vc, bt, lens, 0.4, True, (4, -1))
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert (o[b] == 0).all() and np.isneginf(lse[b]).all()
+            continue
+        ob, lseb = orc.attention_fwd(q[b:b + 1], k[b:b + 1, :n], v[b:b + 1, :n], 0.4, True,
+                                     (4, -1))
+        np.testing.assert_allclose(o[b:b + 1], ob, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b:b + 1], lseb, rtol=0, atol=1e-12)
+
+
 ALL_CHECKS = [check_bruteforce, check_library_fwd, check_golden, check_closed_forms,
               check_invariants, check_mqa_equivalence, check_walkthrough, check_backward,
-              check_empty_rows]
+              check_empty_rows, check_paged]
 
 
 @pytest.fixture(scope="module")
@@ -380,6 +434,17 @@ def test_thread_count_does_not_change_bits(orc):
         np.testing.assert_array_equal(x, y)
 
 
+def test_paged_rejects_bad_page_ids(orc):
+    q, k, v = rand((1, 1, 2, 4), 141), rand((1, 9, 2, 4), 142), rand((1, 9, 2, 4), 143)
+    kc, vc, bt = scatter_to_pages(k, v, 4, 0, 144)
+    bt = bt.copy()
+    bt[0, 1] = kc.shape[0]  # past the last page, inside the sequence
+    with pytest.raises(RuntimeError):
+        orc.attention_fwd_paged(q, kc, vc, bt, [9], 0.5)
+    with pytest.raises(RuntimeError):  # longer than the block table allows
+        orc.attention_fwd_paged(q, kc, vc, bt, [4 * bt.shape[1] + 1], 0.5)
+
+
 def test_rejects_bad_shapes(orc):
     with pytest.raises(ValueError):
         orc.attention_fwd(rand((1, 4, 3, 2), 0), rand((1, 4, 2, 2), 0), rand((1, 4, 2, 2), 0), 1.0)
@@ -405,6 +470,11 @@ MUTATIONS = {
                   "const double* kj = kv_row(c->v, s, b, j, g);\n        for"),
     "one head per kv group in dK": ("for (int h = g * G; h < (g + 1) * G; ++h)",
                                     "for (int h = g * G; h < g * G + 1; ++h)"),
+    "paged row from the page index": ("long row = j % c->P;", "long row = j / c->P;"),
+    "paged last key dropped": ("int nk = c->seqlens[b];",
+                               "int nk = c->seqlens[b] > 0 ? c->seqlens[b] - 1 : 0;"),
+    "paged mask aligned top-left": ("shape_t s = {1, c->Nq, nk,", "shape_t s = {1, c->Nq, c->Nq,"),
+    "paged kv head interleaved": ("int kv_head = h / (c->Hq / c->Hkv);", "int kv_head = h % c->Hkv;"),
 }
 
 
