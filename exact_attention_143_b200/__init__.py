@@ -36,7 +36,8 @@ FA_ERR_DEVICE_TIMEOUT = 6
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
-            "fa_bwd_noalloc", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen")
+            "fa_bwd_noalloc", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
+            "fa_fwd_paged_workspace_size", "fa_fwd_paged")
 
 _lib = None
 
@@ -82,6 +83,11 @@ def load_library(path: str = LIB_PATH):
     lib.fa_bwd_varlen.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.fa_selftest_wait_timeout.restype = i
+    lib.fa_fwd_paged_workspace_size.argtypes = [i] * 8
+    lib.fa_fwd_paged_workspace_size.restype = ctypes.c_size_t
+    lib.fa_fwd_paged.argtypes = ([vp] * 7 + [i] * 8 + [ctypes.c_int64] + [i64p] * 4 +
+                                 [i, f, i, i, i, i, vp, ctypes.c_size_t, vp])
+    lib.fa_fwd_paged.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -311,3 +317,70 @@ def selftest_wait_timeout(limit_ns: int, device=None) -> int:
 
 def set_wait_limit_ns(limit_ns: int) -> int:
     return int(load_library().fa_set_wait_limit_ns(int(limit_ns)))
+
+
+def fa_fwd_paged_workspace_size(B, Nq, Hq, Hkv, d, page_size, max_pages_per_seq, num_splits=0):
+    """Bytes of workspace fa_fwd_paged needs (0 when the keys are not split)."""
+    return int(load_library().fa_fwd_paged_workspace_size(int(B), int(Nq), int(Hq), int(Hkv),
+                                                          int(d), int(page_size),
+                                                          int(max_pages_per_seq),
+                                                          int(num_splits)))
+
+
+def _cache_strides(t: torch.Tensor):
+    if t.dim() != 4:
+        raise ValueError("expected a [num_pages, page_size, kv_heads, head_dim] cache, got shape "
+                         "%s" % (tuple(t.shape),))
+    if t.stride(3) != 1 and t.shape[3] > 1:
+        raise ValueError("head_dim must be contiguous (stride 1)")
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def fa_fwd_paged(q, k_cache, v_cache, block_table, cache_seqlens, softmax_scale=None,
+                 causal=False, window_size=(-1, -1), num_splits=0, out=None, lse=None,
+                 workspace=None):
+    """Decode: q [B, Nq, Hq, d] against a paged KV cache.
+
+    k_cache / v_cache are [num_pages, page_size, Hkv, d]; block_table is int32
+    [B, max_pages_per_seq] (row stride free, entries contiguous) and
+    cache_seqlens int32 [B], both on the device.  The queries are the last Nq
+    positions of each sequence.  Returns (o [B, Nq, Hq, d], lse [B, Hq, Nq])."""
+    lib = load_library()
+    dev = _check_cuda(q, k_cache, v_cache, block_table, cache_seqlens)
+    code = _dtype_code(q)
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise TypeError("q and the caches must share one dtype")
+    if tuple(k_cache.shape) != tuple(v_cache.shape):
+        raise ValueError("k_cache and v_cache must have one shape")
+    B, Nq, Hq, d = q.shape
+    num_pages, page_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B \
+            or block_table.stride(1) != 1:
+        raise ValueError("block_table must be an int32 [B, max_pages] tensor with contiguous rows")
+    if cache_seqlens.dtype != torch.int32 or tuple(cache_seqlens.shape) != (B,) \
+            or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous int32 [B] tensor")
+    max_pages = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Nq, Hq, d), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Nq] tensor")
+    need = fa_fwd_paged_workspace_size(B, Nq, Hq, Hkv, d, page_size, max_pages, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    wl, wr = window_size
+    with torch.cuda.device(dev):
+        rc = lib.fa_fwd_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                              block_table.data_ptr(), cache_seqlens.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), B, Nq, Hq, Hkv, d, page_size, num_pages, max_pages,
+                              block_table.stride(0), _strides(q), _cache_strides(k_cache),
+                              _cache_strides(v_cache), _strides(out), code,
+                              _scale(softmax_scale, d), int(bool(causal)), int(wl), int(wr),
+                              int(num_splits), ws_ptr, ws_bytes, _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_fwd_paged")
+    return out, lse

@@ -13,6 +13,7 @@
 
 #include "fa143.h"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -636,3 +637,240 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                 dk_stride, dv_stride, dtype, softmax_scale, causal, window_left, window_right,
                 stream);
 }
+
+// ------------------------------------------------------------------ paged KV cache (decode)
+namespace {
+
+int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+    else
+      n = 148;
+  });
+  return n;
+}
+
+// Splits of the key tiles of every (sequence, kv head): enough CTAs for about
+// two per SM when the batch alone does not provide them, at least one tile each.
+int decode_splits(int B, int Hkv, int max_tiles, int requested, int& tiles_per_split) {
+  int splits;
+  if (requested > 0) {
+    splits = requested;
+  } else {
+    const int64_t units = int64_t(B) * Hkv;
+    const int64_t want = 2 * int64_t(sm_count());
+    splits = units >= want ? 1 : int((want + units - 1) / units);
+  }
+  splits = std::max(1, std::min(splits, max_tiles));
+  tiles_per_split = (max_tiles + splits - 1) / splits;
+  return (max_tiles + tiles_per_split - 1) / tiles_per_split;
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int check_paged_shape(int B, int Nq, int Hq, int Hkv, int d, int page_size, int num_pages,
+                      int max_pages, int dtype, float scale, int window_left, int window_right) {
+  if (B < 1 || Nq < 1 || Hq < 1 || Hkv < 1 || num_pages < 1 || max_pages < 1)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (window_left < -1 || window_right < -1 || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if ((Hq / Hkv) * Nq > 128) return FA_ERR_UNSUPPORTED;  // one 128-row query tile per kv head
+  if (!is_pow2(page_size) || page_size < 8 || page_size > (1 << 20)) return FA_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535 || num_pages > (1 << 30) ||
+      int64_t(max_pages) * page_size > (int64_t(1) << 30))
+    return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+// 4-D map over a paged cache [num_pages, P, Hkv, d] (innermost first: d, Hkv,
+// P, pages), box of 64 columns x 1 head x min(P, 128) rows x 1 page.
+int make_cache_map(CUtensorMap* map, const void* ptr, const int64_t st[3], int num_pages, int P,
+                   int Hkv, int d, int dtype) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const int64_t sp = num_pages > 1 ? st[0] : 8;
+  const int64_t stok = P > 1 ? st[1] : 8;
+  const int64_t sh = Hkv > 1 ? st[2] : 8;
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(Hkv), cuuint64_t(P), cuuint64_t(num_pages)};
+  cuuint64_t strides[3] = {cuuint64_t(sh) * 2, cuuint64_t(stok) * 2, cuuint64_t(sp) * 2};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(std::min(P, 128)), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map,
+                   dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_ALIGNMENT;
+}
+
+// 4-D map over q [B, Nq, Hq, d] whose box is the whole query tile of one kv
+// head: 64 columns x Nq queries x G heads x 1 sequence (rows h' * Nq + i).
+int make_group_q_map(CUtensorMap* map, const TensorDesc& t, int G, int dtype) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const int64_t ss = t.N > 1 ? t.ss : 8;
+  const int64_t sh = t.H > 1 ? t.sh : 8;
+  const int64_t sb = t.B > 1 ? t.sb : 8;
+  cuuint64_t dims[4] = {cuuint64_t(t.d), cuuint64_t(t.N), cuuint64_t(t.H), cuuint64_t(t.B)};
+  cuuint64_t strides[3] = {cuuint64_t(ss) * 2, cuuint64_t(sh) * 2, cuuint64_t(sb) * 2};
+  cuuint32_t box[4] = {64, cuuint32_t(t.N), cuuint32_t(G), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map,
+                   dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(t.ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_ALIGNMENT;
+}
+
+size_t paged_workspace_bytes(int B, int Hkv, int R, int d, int splits) {
+  if (splits <= 1) return 0;
+  const size_t rows = size_t(B) * Hkv * splits * R;
+  const size_t o_bytes = (rows * d * sizeof(float) + 255) & ~size_t(255);
+  return o_bytes + rows * sizeof(float);
+}
+
+template <int D, bool BF16>
+int launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const fa::DecodeParams& prm, cudaStream_t st) {
+  using Cfg = fa::DecCfg<D>;
+  auto kern = fa::fa_decode_kernel<D, BF16>;
+  static bool attr_done = false;  // per instantiation and process
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+      return FA_ERR_CUDA;
+    attr_done = true;
+  }
+  dim3 grid(unsigned(prm.n_splits), unsigned(prm.Hkv), unsigned(prm.B));
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (prm.n_splits > 1) {
+    const int64_t rows = int64_t(prm.B) * prm.Hq * prm.Nq;
+    fa::fa_decode_combine_kernel<D, BF16><<<unsigned((rows + 3) / 4), 128, 0, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_fwd_paged_workspace_size(int B, int Nq, int Hq, int Hkv, int d, int page_size,
+                                   int max_pages_per_seq, int num_splits) {
+  if (check_paged_shape(B, Nq, Hq, Hkv, d, page_size, 1, max_pages_per_seq, FA_BF16, 1.f, -1,
+                        -1))
+    return 0;
+  const int max_tiles =
+      int((int64_t(max_pages_per_seq) * page_size + 127) / 128);
+  int tps = 0;
+  const int splits = decode_splits(B, Hkv, max_tiles, num_splits, tps);
+  return paged_workspace_bytes(B, Hkv, (Hq / Hkv) * Nq, d, splits);
+}
+
+int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                 const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Hq, int Hkv,
+                 int d, int page_size, int num_pages, int max_pages_per_seq,
+                 int64_t block_table_stride, const int64_t q_stride[3],
+                 const int64_t kcache_stride[3], const int64_t vcache_stride[3],
+                 const int64_t o_stride[3], int dtype, float softmax_scale, int causal,
+                 int window_left, int window_right, int num_splits, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  int rc = check_paged_shape(B, Nq, Hq, Hkv, d, page_size, num_pages, max_pages_per_seq, dtype,
+                             softmax_scale, window_left, window_right);
+  if (rc) return rc;
+  if (!q_stride || !kcache_stride || !vcache_stride || !o_stride || !lse || !block_table ||
+      !cache_seqlens || num_splits < 0)
+    return FA_ERR_INVALID_ARG;
+  if (block_table_stride < max_pages_per_seq) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGNMENT;
+  const int G = Hq / Hkv;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  // the caches as [pages, page_size, Hkv, d] descriptors (batch = page)
+  const TensorDesc tk{k_cache, kcache_stride[0], kcache_stride[1], kcache_stride[2], num_pages,
+                      page_size, Hkv, d};
+  const TensorDesc tv{v_cache, vcache_stride[0], vcache_stride[1], vcache_stride[2], num_pages,
+                      page_size, Hkv, d};
+  for (const TensorDesc* t : {&tq, &to, &tk, &tv})
+    if ((rc = check_tensor(*t))) return rc;
+  const size_t lse_bytes = size_t(B) * Hq * Nq * sizeof(float);
+  if (overlaps_t(to, tq) || overlaps_t(to, tk) || overlaps_t(to, tv) ||
+      overlaps_span(tq, lse, lse_bytes) || overlaps_span(tk, lse, lse_bytes) ||
+      overlaps_span(tv, lse, lse_bytes) || overlaps_span(to, lse, lse_bytes))
+    return FA_ERR_INVALID_ARG;
+
+  const int max_tiles = int((int64_t(max_pages_per_seq) * page_size + 127) / 128);
+  int tps = 0;
+  const int splits = decode_splits(B, Hkv, max_tiles, num_splits, tps);
+  const size_t need = paged_workspace_bytes(B, Hkv, G * Nq, d, splits);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
+    if (overlaps_span(to, workspace, need) || overlaps_span(tq, workspace, need) ||
+        overlaps(reinterpret_cast<uintptr_t>(lse), reinterpret_cast<uintptr_t>(lse) + lse_bytes,
+                 reinterpret_cast<uintptr_t>(workspace),
+                 reinterpret_cast<uintptr_t>(workspace) + need))
+      return FA_ERR_INVALID_ARG;
+  }
+
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_group_q_map(&mq, tq, G, dtype)) ||
+      (rc = make_cache_map(&mk, k_cache, kcache_stride, num_pages, page_size, Hkv, d, dtype)) ||
+      (rc = make_cache_map(&mv, v_cache, vcache_stride, num_pages, page_size, Hkv, d, dtype)))
+    return rc;
+  fa::DecodeParams prm{};
+  prm.block_table = block_table;
+  prm.cache_seqlens = cache_seqlens;
+  prm.bt_stride = block_table_stride;
+  prm.B = B;
+  prm.Nq = Nq;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = G;
+  prm.R = G * Nq;
+  prm.P = page_size;
+  prm.num_pages = num_pages;
+  prm.max_pages = max_pages_per_seq;
+  prm.n_splits = splits;
+  prm.tiles_per_split = tps;
+  prm.scale_log2 = scale_log2_of(softmax_scale);
+  prm.qk_negate = softmax_scale < 0.f ? 1u : 0u;
+  prm.causal = causal ? 1 : 0;
+  prm.wl = window_left;
+  prm.wr = window_right;
+  prm.o = o;
+  prm.o_sb = to.sb;
+  prm.o_ss = to.ss;
+  prm.o_sh = to.sh;
+  prm.lse = lse;
+  if (need > 0) {
+    const size_t rows = size_t(B) * Hkv * splits * G * Nq;
+    prm.part_o = static_cast<float*>(workspace);
+    prm.part_lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                             ((rows * d * sizeof(float) + 255) & ~size_t(255)));
+  }
+  prm.err = device_error_ptr();
+  prm.wait_limit_ns = g_wait_limit_ns;
+  if (!prm.err) return FA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16)
+    return d == 64 ? launch_decode<64, true>(mq, mk, mv, prm, st)
+                   : launch_decode<128, true>(mq, mk, mv, prm, st);
+  return d == 64 ? launch_decode<64, false>(mq, mk, mv, prm, st)
+                 : launch_decode<128, false>(mq, mk, mv, prm, st);
+}
+
+}  // extern "C"

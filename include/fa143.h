@@ -120,6 +120,48 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                   int window_right, void* stream);
 
 /*
+ * Decode against a paged KV cache.
+ *
+ * Sequence b holds cache_seqlens[b] keys; key j of it is row j % page_size of
+ * page block_table[b * block_table_stride + j / page_size] of k_cache and
+ * v_cache ("optimizing-attention-flash", the list of advanced features, which
+ * names a paged KV cache; "FlashAttention V3 原理与…实战指南", section 四 on
+ * inference: the KV cache kept in pages of 16 tokens in its vLLM example).
+ * The Nq queries of sequence b attend to those keys exactly as in fa_fwd, the
+ * masks aligned bottom-right against cache_seqlens[b]: query i is position
+ * cache_seqlens[b] - Nq + i (so with Nq = 1 and causal it sees every key).
+ *   q, o            [B, Nq, Hq, d]            strides {batch, seq, head}
+ *   k_cache, v_cache [num_pages, page_size, Hkv, d] strides {page, token, head}
+ *   block_table     device int32, row b at b * block_table_stride, first
+ *                   ceil(cache_seqlens[b] / page_size) entries used
+ *   cache_seqlens   device int32 [B]
+ *   lse             [B, Hq, Nq] fp32, natural log, contiguous, written
+ *   page_size       a power of two, 8 or more
+ *   num_splits      0 = chosen by the library; k > 0 = the key tiles of each
+ *                   (sequence, kv head) are cut into at most k parts
+ *   workspace       device memory of fa_fwd_paged_workspace_size() bytes,
+ *                   256-byte aligned (may be NULL when that size is 0)
+ * (Hq / Hkv) * Nq must be at most 128.  Lengths are clamped to
+ * [0, max_pages_per_seq * page_size] on the device, and a page id outside
+ * [0, num_pages) reads zeros, so a malformed table gives wrong results but no
+ * access outside the caches.  A sequence with no visible key gets O = 0 and
+ * LSE = -inf.  Inputs are read only; o and lse must not overlap them.
+ * Returns FA_OK once queued, FA_ERR_WORKSPACE if the workspace is missing or
+ * too small, FA_ERR_UNSUPPORTED for dtype, head_dim or a query tile over 128
+ * rows, FA_ERR_ALIGNMENT or FA_ERR_INVALID_ARG as for fa_fwd.
+ */
+size_t fa_fwd_paged_workspace_size(int B, int Nq, int Hq, int Hkv, int d, int page_size,
+                                   int max_pages_per_seq, int num_splits);
+int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* block_table, const int32_t* cache_seqlens, void* o, float* lse,
+                 int B, int Nq, int Hq, int Hkv, int d, int page_size, int num_pages,
+                 int max_pages_per_seq, int64_t block_table_stride,
+                 const int64_t q_stride[3], const int64_t kcache_stride[3],
+                 const int64_t vcache_stride[3], const int64_t o_stride[3], int dtype,
+                 float softmax_scale, int causal, int window_left, int window_right,
+                 int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
  * accumulator [B, Nq, Hq, d] and the fp32 row terms D and LSE*log2(e)
  * [B, Hq, Nq].  The caller allocates it (256-byte aligned); its contents

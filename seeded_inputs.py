@@ -162,3 +162,84 @@ def sample_rows(batch, q_heads, seqlen_q, n, seed):
         i[1] = seqlen_q - 1
     rows = torch.stack([b, h, i], dim=1)
     return torch.unique(rows, dim=0).numpy()
+
+
+@dataclass(frozen=True)
+class PagedWorkload:
+    """Decode: Nq new queries per sequence against a paged KV cache."""
+    name: str
+    n_seqs: int
+    min_len: int
+    max_len: int
+    Nq: int
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    dtype: torch.dtype
+    page_size: int
+    causal: bool
+    seed: int
+
+    @property
+    def softmax_scale(self) -> float:
+        return float(self.head_dim) ** -0.5
+
+    def lengths(self):
+        g = torch.Generator(device="cpu")
+        g.manual_seed(int(self.seed))
+        return [int(x) for x in torch.randint(self.min_len, self.max_len + 1, (self.n_seqs,),
+                                              generator=g)]
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "sequences": self.n_seqs,
+                "cache_lengths": "uniform in [%d, %d]" % (self.min_len, self.max_len),
+                "new_queries": self.Nq, "q_heads": self.q_heads, "kv_heads": self.kv_heads,
+                "head_dim": self.head_dim, "dtype": str(self.dtype).replace("torch.", ""),
+                "page_size": self.page_size, "causal": self.causal, "seed": self.seed}
+
+
+# Decode shape: 128 running sequences and 16-token pages, as in the vLLM launch
+# example of the FlashAttention V3 page (section 四: max_num_seqs=128,
+# block_size=16); 32 query heads over 8 kv heads of dimension 128 (the
+# geometry of the Llama-3-8B model that example serves).
+PAGED_WORKLOADS = {
+    "decode_128seq_512to8192_h32kv8_d128_bf16_page16": PagedWorkload(
+        "decode_128seq_512to8192_h32kv8_d128_bf16_page16", 128, 512, 8192, 1, 32, 8, 128, BF16,
+        16, True, seed=6),
+}
+
+
+def make_paged_inputs(B, Nq, Hq, Hkv, d, dtype, page_size, lens, seed, spare_pages=3,
+                      fill=float("nan")):
+    """q [B, Nq, Hq, d] and a paged cache holding len_b keys per sequence.
+
+    Returns q, k_cache, v_cache ([num_pages, page_size, Hkv, d]), block_table
+    (int32 [B, max_pages]) and cache_seqlens (int32 [B]), all on the CPU.
+    Pages are handed out in a seeded random order; cache rows a sequence does
+    not own (past its length, and `spare_pages` unused pages) hold `fill`.
+    Draw order: q, then per sequence its K rows and V rows."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    n_pages_of = [(n + page_size - 1) // page_size for n in lens]
+    max_pages = max(1, max(n_pages_of))
+    num_pages = sum(n_pages_of) + spare_pages
+    q = torch.randn((B, Nq, Hq, d), generator=g, dtype=torch.float32).to(dtype)
+    perm = torch.randperm(max(num_pages, 1), generator=g)
+    k_cache = torch.full((max(num_pages, 1), page_size, Hkv, d), fill, dtype=dtype)
+    v_cache = torch.full((max(num_pages, 1), page_size, Hkv, d), fill, dtype=dtype)
+    block_table = torch.zeros((B, max_pages), dtype=torch.int32)
+    k_rows = k_cache.view(-1, Hkv, d)  # row p * page_size + t of page p
+    v_rows = v_cache.view(-1, Hkv, d)
+    first = 0
+    for b, n in enumerate(lens):
+        pages = perm[first:first + n_pages_of[b]]
+        first += n_pages_of[b]
+        block_table[b, :len(pages)] = pages.to(torch.int32)
+        kk = torch.randn((n, Hkv, d), generator=g, dtype=torch.float32).to(dtype)
+        vv = torch.randn((n, Hkv, d), generator=g, dtype=torch.float32).to(dtype)
+        j = torch.arange(n)
+        rows = pages[j // page_size] * page_size + j % page_size
+        k_rows[rows] = kk
+        v_rows[rows] = vv
+    cache_seqlens = torch.tensor(lens, dtype=torch.int32)
+    return q, k_cache, v_cache, block_table, cache_seqlens
