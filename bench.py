@@ -37,8 +37,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from seeded_inputs import (VARLEN_WORKLOADS, WORKLOADS, Workload, make_qkv,  # noqa: E402
-                           make_varlen_inputs, make_workload_inputs)
+from seeded_inputs import (PAGED_WORKLOADS, VARLEN_WORKLOADS, WORKLOADS, Workload,  # noqa: E402
+                           make_paged_inputs, make_qkv, make_varlen_inputs,
+                           make_workload_inputs)
 
 METRIC = "attention TFLOPS (fwd, fwd+bwd) on 1 B200 and % of dense FP16/BF16 tensor peak"
 MAIN_WORKLOAD = "fwdbwd_1x16384_h16_d128_bf16_causal"
@@ -387,6 +388,35 @@ def run_ours(args):
                               "bwd_ms_median": round(bm_v, 4),
                               "bwd_tflops": round(2.5 * vf / (bm_v / 1e3) / 1e12, 1)}
             del vq, vk, vv, vdo, vo, vl, vws, vdq, vdk, vdv
+        # decode against a paged KV cache: bound by HBM, reported in GB/s of
+        # algorithmic traffic (every cached K and V row of every sequence read
+        # once, q read and o, lse written once)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        for pw in PAGED_WORKLOADS.values():
+            plens = pw.lengths()
+            pq, pkc, pvc, pbt, psl = (t.to(dev) for t in make_paged_inputs(
+                pw.n_seqs, pw.Nq, pw.q_heads, pw.kv_heads, pw.head_dim, pw.dtype, pw.page_size,
+                plens, pw.seed))
+            po = torch.empty_like(pq)
+            pl = torch.empty(pw.n_seqs, pw.q_heads, pw.Nq, dtype=torch.float32, device=dev)
+            pneed = fa.fa_fwd_paged_workspace_size(pw.n_seqs, pw.Nq, pw.q_heads, pw.kv_heads,
+                                                   pw.head_dim, pw.page_size, pbt.shape[1])
+            pws = torch.empty(max(pneed, 256), dtype=torch.uint8, device=dev)
+            pkw = dict(softmax_scale=pw.softmax_scale, causal=pw.causal)
+            pms = time_steps(lambda _: fa.fa_fwd_paged(pq, pkc, pvc, pbt, psl, out=po, lse=pl,
+                                                       workspace=pws, **pkw), 20, 3, flush, stream)
+            pm = statistics.median(pms)
+            kv_bytes = 2 * sum(plens) * pw.kv_heads * pw.head_dim * pkc.element_size()
+            io_bytes = (2 * pq.numel() * pq.element_size() + pl.numel() * 4 + psl.numel() * 4 +
+                        sum((n + pw.page_size - 1) // pw.page_size for n in plens) * 4)
+            gbs = (kv_bytes + io_bytes) / (pm / 1e3) / 1e9
+            table[pw.name] = {"cached_tokens": sum(plens), "ms_median": round(pm, 4),
+                              "ms_min": round(min(pms), 4),
+                              "algorithmic_bytes": kv_bytes + io_bytes,
+                              "gb_per_s": round(gbs, 1), "hbm_peak_gb_per_s": hbm,
+                              "frac_of_hbm": round(gbs / hbm, 4),
+                              "decode_tokens_per_s": round(pw.n_seqs * pw.Nq / (pm / 1e3), 1)}
+            del pq, pkc, pvc, pbt, psl, po, pl, pws
         # the main workload's forward and backward separately
         fms = time_steps(lambda _: fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw), 10, 3, flush,
                          stream)

@@ -22,9 +22,9 @@
 //   rows: the G query heads of kv head g times the Nq queries (r = h' Nq + i)
 //   form one 128-row tile (rows past G Nq are zero), loaded by one TMA box.
 //   warp 4   TMA: the query tile once, then a ring of K and V tiles, each
-//            assembled from 128 / min(P, 128) page boxes; a page past the
-//            sequence is fetched at an out-of-range page coordinate, which
-//            TMA fills with zeros.
+//            assembled from 128 / min(P, 128) page boxes issued by as many
+//            lanes; a page past the sequence is fetched at an out-of-range
+//            page coordinate, which TMA fills with zeros.
 //   warp 5   tcgen05 issuer: S = Q K^T into one of two tensor-memory
 //            regions, O += P V with P read from tensor memory (as in the
 //            forward kernel).
@@ -164,38 +164,50 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(bar_q, uint32_t(p.R * 128 * (D / 64)));
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_4d(sbase + Cfg::kSmemQ + c * Cfg::kChunk, &tmQ, bar_q, c * 64, 0, g * p.G, b);
+    // The whole warp runs the loop.  Lane bx reads the page id of box bx of
+    // the tile before the wait for the free stage and then issues that box's
+    // copies, so the copies of one tile leave from up to 16 threads.
+    if (n > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        mbar_arrive_expect_tx(bar_q, uint32_t(p.R * 128 * (D / 64)));
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sbase + Cfg::kSmemQ + c * Cfg::kChunk, &tmQ, bar_q, c * 64, 0, g * p.G, b);
+      }
       const int rows_per_box = min(p.P, 128);
-      const int boxes = 128 / rows_per_box;
+      const int boxes = 128 / rows_per_box;  // at most 16 (pages of 8 or more rows)
       const int* bt = p.block_table + int64_t(b) * p.bt_stride;
       const int n_seq_pages = (Nk + p.P - 1) / p.P;
       bool ok = true;
       for (int jj = 0; jj < n && ok; ++jj) {
         const int s = jj % S, u = jj / S;
-        if (u > 0 && !(ok = mbar_wait(bar_empty(s), (u - 1) & 1, wc))) break;
-        mbar_arrive_expect_tx(bar_full(s), 2 * Cfg::kTileBytes);
         const int key0 = (j0 + jj) * 128;
-        for (int bx = 0; bx < boxes; ++bx) {
-          const int key = key0 + bx * rows_per_box;
-          const int pg = key / p.P;
-          // a page the sequence does not hold is read at an out-of-range page
-          // coordinate: TMA delivers zeros for it
-          const int page = pg < n_seq_pages ? bt[pg] : p.num_pages;
-          const int tok = key % p.P;
-          const uint32_t row_off = uint32_t(bx * rows_per_box * 128);
+        // a page the sequence does not hold is read at an out-of-range page
+        // coordinate: TMA delivers zeros for it
+        int my_page = p.num_pages;
+        if (lane < boxes) {
+          const int pg = (key0 + lane * rows_per_box) / p.P;
+          if (pg < n_seq_pages) my_page = bt[pg];
+        }
+        if (u > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_empty(s), (u - 1) & 1, wc));
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(bar_full(s), 2 * Cfg::kTileBytes);
+        __syncwarp();
+        // lane bx copies the boxes of its own page: a single issuing thread
+        // cannot keep the copy engine busy with boxes this small
+        if (lane < boxes) {
+          const int tok = (key0 + lane * rows_per_box) % p.P;
+          const uint32_t row_off = uint32_t(lane * rows_per_box * 128);
           for (int c = 0; c < D / 64; ++c) {
             tma_load_4d(sbase + Cfg::kSmemK + s * Cfg::kTileBytes + c * Cfg::kChunk + row_off,
-                        &tmK, bar_full(s), c * 64, g, tok, page);
+                        &tmK, bar_full(s), c * 64, g, tok, my_page);
             tma_load_4d(sbase + Cfg::kSmemV + s * Cfg::kTileBytes + c * Cfg::kChunk + row_off,
-                        &tmV, bar_full(s), c * 64, g, tok, page);
+                        &tmV, bar_full(s), c * 64, g, tok, my_page);
           }
         }
+        __syncwarp();
       }
     }
   } else if (warp == 5) {
