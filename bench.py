@@ -37,9 +37,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from seeded_inputs import (PAGED_WORKLOADS, VARLEN_WORKLOADS, WORKLOADS, Workload,  # noqa: E402
-                           make_paged_inputs, make_qkv, make_varlen_inputs,
-                           make_workload_inputs)
+from seeded_inputs import (FP8_WORKLOADS, PAGED_WORKLOADS, VARLEN_WORKLOADS,  # noqa: E402
+                           WORKLOADS, Workload, make_fp8_inputs, make_paged_inputs, make_qkv,
+                           make_varlen_inputs, make_workload_inputs)
 
 METRIC = "attention TFLOPS (fwd, fwd+bwd) on 1 B200 and % of dense FP16/BF16 tensor peak"
 MAIN_WORKLOAD = "fwdbwd_1x16384_h16_d128_bf16_causal"
@@ -417,6 +417,28 @@ def run_ours(args):
                               "frac_of_hbm": round(gbs / hbm, 4),
                               "decode_tokens_per_s": round(pw.n_seqs * pw.Nq / (pm / 1e3), 1)}
             del pq, pkc, pvc, pbt, psl, po, pl, pws
+        # FP8 (e4m3) forward: counted FLOPs over the e4m3 tensor peak, taken as
+        # the measured bf16 rate times the nominal fp8 / bf16 ratio of 2
+        for fw in FP8_WORKLOADS.values():
+            fq, fk, fv = (t.to(dev) for t in make_fp8_inputs(
+                fw.batch, fw.seqlen, fw.seqlen, fw.q_heads, fw.kv_heads, fw.head_dim,
+                fw.descales, fw.seed))
+            fo = torch.empty(fq.shape, dtype=torch.bfloat16, device=dev)
+            fl = torch.empty(fw.batch, fw.q_heads, fw.seqlen, dtype=torch.float32, device=dev)
+            fkw = dict(softmax_scale=fw.softmax_scale, causal=fw.causal,
+                       descale_q=fw.descales[0], descale_k=fw.descales[1],
+                       descale_v=fw.descales[2])
+            fms8 = time_steps(lambda _: fa.fa_fwd_fp8(fq, fk, fv, out=fo, lse=fl, **fkw), 20, 3,
+                              flush, stream)
+            fm8 = statistics.median(fms8)
+            ff = 4.0 * fw.batch * fw.q_heads * fw.head_dim * visible_pairs(
+                fw.seqlen, fw.seqlen, fw.causal, (-1, -1))
+            tf8 = ff / (fm8 / 1e3) / 1e12
+            table[fw.name] = {"fwd_ms_median": round(fm8, 4), "fwd_ms_min": round(min(fms8), 4),
+                              "fwd_tflops": round(tf8, 1), "fp8_peak_tflops": 2 * peak,
+                              "frac_of_fp8_peak": round(tf8 / (2 * peak), 4),
+                              "frac_of_bf16_peak": round(tf8 / peak, 4)}
+            del fq, fk, fv, fo, fl
         # the main workload's forward and backward separately
         fms = time_steps(lambda _: fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw), 10, 3, flush,
                          stream)

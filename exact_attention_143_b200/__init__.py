@@ -37,7 +37,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
             "fa_bwd_noalloc", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
-            "fa_fwd_paged_workspace_size", "fa_fwd_paged")
+            "fa_fwd_paged_workspace_size", "fa_fwd_paged", "fa_fwd_fp8")
 
 _lib = None
 
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_paged.argtypes = ([vp] * 7 + [i] * 8 + [ctypes.c_int64] + [i64p] * 4 +
                                  [i, f, i, i, i, i, vp, ctypes.c_size_t, vp])
     lib.fa_fwd_paged.restype = i
+    lib.fa_fwd_fp8.argtypes = [vp] * 5 + [i] * 6 + [i64p] * 4 + [f] * 4 + [i, i, i, vp]
+    lib.fa_fwd_fp8.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -383,4 +385,35 @@ def fa_fwd_paged(q, k_cache, v_cache, block_table, cache_seqlens, softmax_scale=
                               int(num_splits), ws_ptr, ws_bytes, _stream(dev))
     if rc:
         raise FAError(rc, "fa_fwd_paged")
+    return out, lse
+
+
+def fa_fwd_fp8(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), descale_q=1.0,
+               descale_k=1.0, descale_v=1.0, out=None, lse=None):
+    """Forward on float8_e4m3fn q, k, v [B, N, H, d]; returns (o bf16 [B,Nq,Hq,d],
+    lse fp32 [B,Hq,Nq]) for attention of (descale_q q, descale_k k, descale_v v)."""
+    lib = load_library()
+    dev = _check_cuda(q, k, v)
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError("q, k, v must be float8_e4m3fn (got %s)" % t.dtype)
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=dev)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("the FP8 forward writes a bf16 output")
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Nq] tensor")
+    wl, wr = window_size
+    with torch.cuda.device(dev):
+        rc = lib.fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            lse.data_ptr(), B, Nq, Nk, Hq, Hkv, d, _strides(q), _strides(k),
+                            _strides(v), _strides(out), float(descale_q), float(descale_k),
+                            float(descale_v), _scale(softmax_scale, d), int(bool(causal)),
+                            int(wl), int(wr), _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_fwd_fp8")
     return out, lse

@@ -15,6 +15,7 @@
 #include "fa_bwd.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_fp8.cuh"
 
 namespace {
 
@@ -871,6 +872,132 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
                    : launch_decode<128, true>(mq, mk, mv, prm, st);
   return d == 64 ? launch_decode<64, false>(mq, mk, mv, prm, st)
                  : launch_decode<128, false>(mq, mk, mv, prm, st);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ FP8 (e4m3) forward
+namespace {
+
+// An e4m3 tensor [B, N, H, d]: one byte per element, so strides (in
+// elements) must be multiples of 16 for the 16-byte TMA rule.
+int check_tensor_fp8(const TensorDesc& t) {
+  if (t.ptr == nullptr) return FA_ERR_INVALID_ARG;
+  if (t.sb < 0 || t.ss < 0 || t.sh < 0) return FA_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return FA_ERR_ALIGNMENT;
+  if ((t.B > 1 && t.sb % 16) || (t.N > 1 && t.ss % 16) || (t.H > 1 && t.sh % 16))
+    return FA_ERR_ALIGNMENT;
+  return FA_OK;
+}
+
+void tensor_extent_bytes(const TensorDesc& t, int elem, uintptr_t& lo, uintptr_t& hi) {
+  const int64_t last = int64_t(t.B - 1) * t.sb + int64_t(t.N - 1) * t.ss +
+                       int64_t(t.H - 1) * t.sh + t.d;
+  lo = reinterpret_cast<uintptr_t>(t.ptr);
+  hi = lo + uintptr_t(last) * uintptr_t(elem);
+}
+
+// 4-D map over an e4m3 [B, N, H, d] tensor, box of d columns x 128 rows, with
+// the 128-byte (d = 128) or 64-byte (d = 64) swizzle of one row.
+int make_map_fp8(CUtensorMap* map, const TensorDesc& t) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const int64_t ss = t.N > 1 ? t.ss : 16;
+  const int64_t sh = t.H > 1 ? t.sh : 16;
+  const int64_t sb = t.B > 1 ? t.sb : 16;
+  cuuint64_t dims[4] = {cuuint64_t(t.d), cuuint64_t(t.N), cuuint64_t(t.H), cuuint64_t(t.B)};
+  cuuint64_t strides[3] = {cuuint64_t(ss), cuuint64_t(sh), cuuint64_t(sb)};
+  cuuint32_t box[4] = {cuuint32_t(t.d), 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(t.ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   t.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_ALIGNMENT;
+}
+
+template <int D>
+int launch_fwd_fp8(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const fa::Fp8Params& prm, cudaStream_t st) {
+  using Cfg = fa::Fp8Cfg<D>;
+  auto kern = fa::fa_fwd_fp8_kernel<D>;
+  static bool attr_done = false;  // per instantiation and process
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+      return FA_ERR_CUDA;
+    attr_done = true;
+  }
+  dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+               int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3],
+               const int64_t k_stride[3], const int64_t v_stride[3], const int64_t o_stride[3],
+               float descale_q, float descale_k, float descale_v, float softmax_scale,
+               int causal, int window_left, int window_right, void* stream) {
+  // dtype argument of the 16-bit checks: the output is bf16
+  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, FA_BF16, softmax_scale, window_left,
+                        window_right);
+  if (rc) return rc;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v))
+    return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  for (const TensorDesc* t : {&tq, &tk, &tv})
+    if ((rc = check_tensor_fp8(*t))) return rc;
+  if ((rc = check_tensor(to))) return rc;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_ALIGNMENT;
+  const size_t lse_bytes = size_t(B) * Hq * Nq * sizeof(float);
+  uintptr_t o0, o1, l0 = reinterpret_cast<uintptr_t>(lse), l1 = l0 + lse_bytes;
+  tensor_extent(to, o0, o1);
+  for (const TensorDesc* t : {&tq, &tk, &tv}) {
+    uintptr_t a0, a1;
+    tensor_extent_bytes(*t, 1, a0, a1);
+    if (overlaps(a0, a1, o0, o1) || overlaps(a0, a1, l0, l1)) return FA_ERR_INVALID_ARG;
+  }
+  if (overlaps(o0, o1, l0, l1)) return FA_ERR_INVALID_ARG;
+
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_map_fp8(&mq, tq)) || (rc = make_map_fp8(&mk, tk)) ||
+      (rc = make_map_fp8(&mv, tv)))
+    return rc;
+  fa::Fp8Params prm{};
+  prm.o = o;
+  prm.lse = lse;
+  prm.o_sb = to.sb;
+  prm.o_ss = to.ss;
+  prm.o_sh = to.sh;
+  prm.B = B;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.n_mblocks = (Nq + 255) / 256;
+  // the dequantisation factors of Q and K scale every score; a negative
+  // product flips the sign of Q K^T like a negative softmax scale
+  const float qk = softmax_scale * descale_q * descale_k;
+  prm.scale_log2 = scale_log2_of(qk);
+  prm.qk_negate = qk < 0.f ? 1u : 0u;
+  prm.out_scale = descale_v;
+  prm.causal = causal ? 1 : 0;
+  prm.wl = window_left;
+  prm.wr = window_right;
+  prm.err = device_error_ptr();
+  prm.wait_limit_ns = g_wait_limit_ns;
+  if (!prm.err) return FA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd_fp8<64>(mq, mk, mv, prm, st)
+                 : launch_fwd_fp8<128>(mq, mk, mv, prm, st);
 }
 
 }  // extern "C"

@@ -120,6 +120,24 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                   int window_right, void* stream);
 
 /*
+ * Forward on FP8 inputs: q, k, v hold float8_e4m3fn values (one byte each;
+ * "optimizing-attention-flash", Workflow 3: inputs cast to float8_e4m3fn and
+ * passed to the same attention call), o is bf16, lse fp32 [B, Hq, Nq].
+ * The result is exact attention of (descale_q q, descale_k k, descale_v v)
+ * with the masks and GQA mapping of fa_fwd.  S = Q K^T is exact in fp32; for
+ * P V the probabilities are rounded to e4m3 (held as 2^6 exp(s - m), at most
+ * 256), so each term of O carries a relative error of at most 2^-4, or an
+ * absolute error of at most 2^-16 where P < 2^-12.  Strides are in elements;
+ * q, k and v strides must be multiples of 16 (16 bytes), o strides multiples
+ * of 8.  d is 64 or 128.  Returns as fa_fwd.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+               int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3],
+               const int64_t k_stride[3], const int64_t v_stride[3], const int64_t o_stride[3],
+               float descale_q, float descale_k, float descale_v, float softmax_scale,
+               int causal, int window_left, int window_right, void* stream);
+
+/*
  * Decode against a paged KV cache.
  *
  * Sequence b holds cache_seqlens[b] keys; key j of it is row j % page_size of

@@ -243,3 +243,52 @@ def make_paged_inputs(B, Nq, Hq, Hkv, d, dtype, page_size, lens, seed, spare_pag
         v_rows[rows] = vv
     cache_seqlens = torch.tensor(lens, dtype=torch.int32)
     return q, k_cache, v_cache, block_table, cache_seqlens
+
+
+@dataclass(frozen=True)
+class Fp8Workload:
+    """Forward on float8_e4m3fn inputs (optionally quantised with per-tensor
+    factors: the stored value is x / descale)."""
+    name: str
+    batch: int
+    seqlen: int
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    causal: bool
+    descales: tuple
+    seed: int
+
+    @property
+    def softmax_scale(self) -> float:
+        return float(self.head_dim) ** -0.5
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "batch": self.batch, "seqlen_q": self.seqlen,
+                "seqlen_k": self.seqlen, "q_heads": self.q_heads, "kv_heads": self.kv_heads,
+                "head_dim": self.head_dim, "dtype": "float8_e4m3fn in, bfloat16 out",
+                "causal": self.causal, "descales": list(self.descales), "seed": self.seed}
+
+
+# The pages' FP8 example shape ("optimizing-attention-flash", Workflow 3,
+# Step 3: 2 x 4096 tokens, 32 heads of 64, cast straight to float8_e4m3fn),
+# and the 16384-token causal d = 128 shape of the 16-bit benchmark.
+FP8_WORKLOADS = {
+    "fwd_fp8_2x4096_h32_d64_e4m3": Fp8Workload("fwd_fp8_2x4096_h32_d64_e4m3", 2, 4096, 32, 32, 64,
+                                               False, (1.0, 1.0, 1.0), seed=7),
+    "fwd_fp8_1x16384_h16_d128_e4m3_causal": Fp8Workload(
+        "fwd_fp8_1x16384_h16_d128_e4m3_causal", 1, 16384, 16, 16, 128, True, (1.0, 1.0, 1.0),
+        seed=8),
+}
+
+
+def make_fp8_inputs(B, Nq, Nk, Hq, Hkv, d, descales, seed):
+    """float8_e4m3fn q [B,Nq,Hq,d], k, v [B,Nk,Hkv,d] on the CPU: seeded N(0,1)
+    fp32 draws in the order Q, K, V, each divided by its descale factor and
+    cast (round to nearest, as torch's cast does)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((B, Nq, Hq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, Nk, Hkv, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Nk, Hkv, d), generator=g, dtype=torch.float32)
+    return tuple((x / float(s)).to(torch.float8_e4m3fn) for x, s in zip((q, k, v), descales))
