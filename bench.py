@@ -44,7 +44,8 @@ from seeded_inputs import (FP8_WORKLOADS, PAGED_WORKLOADS, VARLEN_WORKLOADS,  # 
 METRIC = "attention TFLOPS (fwd, fwd+bwd) on 1 B200 and % of dense FP16/BF16 tensor peak"
 MAIN_WORKLOAD = "fwdbwd_1x16384_h16_d128_bf16_causal"
 FWD_TABLE = ["fwd_2x2048_h8_d64_fp16", "fwd_2x2048_h8_d64_fp16_causal",
-             "fwd_4x4096_h32_d64_fp16_causal", "fwd_2x4096_h32kv8_d128_bf16_causal_win256"]
+             "fwd_4x4096_h32_d64_fp16_causal", "fwd_2x4096_h32kv8_d128_bf16_causal_win256",
+             "fwd_2x4096_h16_d256_bf16_causal"]
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 L2_FLUSH_BYTES = 256 << 20
 

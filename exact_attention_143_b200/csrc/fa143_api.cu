@@ -15,6 +15,7 @@
 #include "fa_bwd.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd256.cuh"
 #include "fa_fwd_fp8.cuh"
 
 namespace {
@@ -90,13 +91,14 @@ bool overlaps_span(const TensorDesc& a, const void* p, size_t bytes) {
 }
 
 int check_common(int B, int Nq, int Nk, int Hq, int Hkv, int d, int dtype, float scale,
-                 int window_left, int window_right) {
+                 int window_left, int window_right, bool allow_d256 = false) {
   if (B < 1 || Nq < 1 || Nk < 1 || Hq < 1 || Hkv < 1) return FA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (window_left < -1 || window_right < -1) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow_d256 && d == 256)) return FA_ERR_UNSUPPORTED;
+  if (d == 256 && (Nq + 127) / 128 > 65535) return FA_ERR_INVALID_ARG;
   // grid and TMA coordinate limits
   if (Nq > (1 << 24) || Nk > (1 << 24) || int64_t(B) * Hq > (int64_t(1) << 30) ||
       (Nq + 255) / 256 > 65535 || (Nk + 127) / 128 > 65535)
@@ -106,7 +108,7 @@ int check_common(int B, int Nq, int Nk, int Hq, int Hkv, int d, int dtype, float
 
 // 4-D tensor map over [B, N, H, d] (innermost first: d, N, H, B), box of
 // 64 columns x 128 rows, 128-byte swizzle, zero fill outside the tensor.
-int make_map(CUtensorMap* map, const TensorDesc& t, int dtype) {
+int make_map(CUtensorMap* map, const TensorDesc& t, int dtype, int box_rows = 128) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return FA_ERR_CUDA;
   // strides of size-1 dimensions are never used; give them a legal value
@@ -115,7 +117,7 @@ int make_map(CUtensorMap* map, const TensorDesc& t, int dtype) {
   const int64_t sb = t.B > 1 ? t.sb : 8;
   cuuint64_t dims[4] = {cuuint64_t(t.d), cuuint64_t(t.N), cuuint64_t(t.H), cuuint64_t(t.B)};
   cuuint64_t strides[3] = {cuuint64_t(ss) * 2, cuuint64_t(sh) * 2, cuuint64_t(sb) * 2};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, cuuint32_t(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map,
                    dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -161,6 +163,23 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
                const fa::FwdParams& prm, cudaStream_t st) {
   using Cfg = fa::FwdCfg<D>;
   auto kern = fa::fa_fwd_kernel<D, BF16>;
+  static bool attr_done = false;  // per instantiation and process
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+      return FA_ERR_CUDA;
+    attr_done = true;
+  }
+  dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool BF16>
+int launch_fwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const fa::FwdParams& prm, cudaStream_t st) {
+  using Cfg = fa::Fwd256Cfg;
+  auto kern = fa::fa_fwd256_kernel<BF16>;
   static bool attr_done = false;  // per instantiation and process
   if (!attr_done) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -272,9 +291,11 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
       overlaps_span(tv, lse, lse_bytes) || overlaps_span(to, lse, lse_bytes))
     return FA_ERR_INVALID_ARG;
 
+  // d = 256 streams K and V in tiles of 64 keys
+  const int kv_rows = d == 256 ? 64 : 128;
   CUtensorMap mq, mk, mv;
-  if ((rc = make_map(&mq, tq, dtype)) || (rc = make_map(&mk, tk, dtype)) ||
-      (rc = make_map(&mv, tv, dtype)))
+  if ((rc = make_map(&mq, tq, dtype)) || (rc = make_map(&mk, tk, dtype, kv_rows)) ||
+      (rc = make_map(&mv, tv, dtype, kv_rows)))
     return rc;
   fa::FwdParams prm{};
   prm.o = const_cast<void*>(to.ptr);
@@ -287,7 +308,7 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   prm.Nk = Nk;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
-  prm.n_mblocks = (Nq + 255) / 256;
+  prm.n_mblocks = d == 256 ? (Nq + 127) / 128 : (Nq + 255) / 256;
   prm.scale_log2 = scale_log2_of(softmax_scale);
   prm.qk_negate = softmax_scale < 0.f ? 1u : 0u;
   prm.causal = causal ? 1 : 0;
@@ -301,6 +322,9 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   prm.total_k = total_k;
   if (!prm.err) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 256)
+    return dtype == FA_BF16 ? launch_fwd256<true>(mq, mk, mv, prm, st)
+                            : launch_fwd256<false>(mq, mk, mv, prm, st);
   if (dtype == FA_BF16)
     return d == 64 ? launch_fwd<64, true>(mq, mk, mv, prm, st)
                    : launch_fwd<128, true>(mq, mk, mv, prm, st);
@@ -326,7 +350,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3], const int64_t k_stride[3],
            const int64_t v_stride[3], const int64_t o_stride[3], int dtype, float softmax_scale,
            int causal, int window_left, int window_right, void* stream) {
-  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right,
+                        true);
   if (rc) return rc;
   if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
   const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
@@ -346,7 +371,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                   float softmax_scale, int causal, int window_left, int window_right,
                   void* stream) {
   int rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale,
-                        window_left, window_right);
+                        window_left, window_right, true);
   if (rc) return rc;
   if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
                          total_k)))

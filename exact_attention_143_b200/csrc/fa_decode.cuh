@@ -26,10 +26,12 @@
 //            lanes; a page past the sequence is fetched at an out-of-range
 //            page coordinate, which TMA fills with zeros.
 //   warp 5   tcgen05 issuer: S = Q K^T into one of two tensor-memory
-//            regions, O += P V with P read from tensor memory (as in the
-//            forward kernel).
+//            regions, O += P V with P read from one of two regions of its own.
 //   warps 0-3 softmax: thread r owns row r (tensor-memory lane r); masks,
-//            running max / sum with the lazy O rescale, P written over S.
+//            running max / sum with the lazy O rescale.  P(j) is written once
+//            P V(j-2), the last reader of its region, is done, and O is
+//            rescaled once P V(j-1) is done, each awaited on the barrier
+//            committed with that MMA.
 //            Thread r also clears V row r of the tile when its key lies past
 //            the cache length: a partly filled page holds whatever the caller
 //            left there, and 0 * NaN would poison O.
@@ -76,6 +78,7 @@ struct DecCfg {
   static constexpr int kSmemBytes = kSmemV + kStages * kTileBytes + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
+  static constexpr uint32_t kColP = 256 + D;  // P(j) at kColP + 64 (j % 2)
 };
 
 // Visible key range [lo, hi] of query i of a sequence holding Nk keys.
@@ -104,7 +107,7 @@ __global__ void __launch_bounds__(192, 1)
   auto bar_empty = [&](int s) { return smem_u32(&bars[1 + S + s]); };  // S_j and P_j V_j done
   auto bar_sfull = [&](int r) { return smem_u32(&bars[1 + 2 * S + r]); };
   auto bar_pfull = [&](int r) { return smem_u32(&bars[3 + 2 * S + r]); };
-  const uint32_t bar_odone = smem_u32(&bars[5 + 2 * S]);
+  auto bar_odone = [&](int r) { return smem_u32(&bars[5 + 2 * S + r]); };  // P V(j), r = j % 2
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
 
@@ -140,8 +143,8 @@ __global__ void __launch_bounds__(192, 1)
     for (int r = 0; r < 2; ++r) {
       mbar_init(bar_sfull(r), 1);
       mbar_init(bar_pfull(r), 128);
+      mbar_init(bar_odone(r), 1);
     }
-    mbar_init(bar_odone, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -212,9 +215,8 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    // S_j goes to region j % 2.  S_{j+2} is issued after P_j V_j, which it
-    // overwrites in the in-order tensor pipe, so two S tiles run ahead of the
-    // softmax.
+    // S_j goes to region j % 2 and P_j to P region j % 2; S_{j+2} is issued
+    // after P_j V_j, so two S tiles run ahead of the softmax.
     if (n > 0) {
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
@@ -253,9 +255,9 @@ __global__ void __launch_bounds__(192, 1)
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts(tmem + Cfg::kColO, tmem + (jj & 1) * 128 + kk * 8,
+            mma_ts(tmem + Cfg::kColO, tmem + Cfg::kColP + (jj & 1) * 64 + kk * 8,
                    vb + uint64_t((kk * 16 * 128) >> 4), idesc_pv, (kk > 0 || jj > 0) ? 1u : 0u);
-          mma_commit(bar_odone);
+          mma_commit(bar_odone(jj & 1));
           mma_commit(bar_empty(s));
         }
         __syncwarp();
@@ -343,6 +345,13 @@ __global__ void __launch_bounds__(192, 1)
         const float2 nb2 = make_float2(-base, -base);
         float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
+        // P(j) replaces P(j-2) once P V(j-2) is done
+        if (jj >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(jj & 1), ((jj >> 1) + 1) & 1, wc));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint32_t tP = tmem + lane_base + Cfg::kColP + (jj & 1) * 64;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -354,14 +363,15 @@ __global__ void __launch_bounds__(192, 1)
             lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);
             pk[c] = pack2<BF16>(pv.x, pv.y);
           }
-          tmem_st32(tS + 32 * half, pk);  // P over S columns already read
+          tmem_st32(tP + 32 * half, pk);
         }
         const float2 ls2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
         l += ls2.x + ls2.y;
       }
       if (jj > 0 && __any_sync(0xffffffffu, grow)) {
         // P_{j-1} V_{j-1} must be in O before it is rescaled
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_odone, (jj - 1) & 1, wc));
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar_odone((jj - 1) & 1), ((jj - 1) >> 1) & 1, wc));
         if (!ok) break;
         tc_fence_after();
         const uint32_t tO = tmem + lane_base + Cfg::kColO;
@@ -380,7 +390,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(bar_pfull(jj & 1));
     }
     // epilogue: this split's O / l and its log2-sum-exp2, or the final O, LSE
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_odone, (n - 1) & 1, wc));
+    // every P V done: the last two, one per region (earlier ones were awaited)
+    for (int jl = max(0, n - 2); jl < n && ok; ++jl)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(jl & 1), (jl >> 1) & 1, wc));
     if (ok && warp_has_rows) {
       tc_fence_after();
       const bool has = (n > 0) && (l > 0.f);

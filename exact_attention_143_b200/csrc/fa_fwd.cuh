@@ -489,9 +489,10 @@ __global__ void __launch_bounds__(352, 1)
           lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);
           pk[c] = pack2<BF16>(pv.x, pv.y);
         }
-        // P_t V_{j-1} must be complete before P_t is rewritten (with P over S
-        // this is implied: S_t(j) itself followed P_t V_{j-1} in the pipe)
-        if (kSepP && half == 0 && jj > 0) {
+        // P_t V_{j-1}, the last reader of P_t, must be complete before P_t is
+        // rewritten.  It is awaited on its own barrier: the completion of
+        // S_t(j), issued after it, does not imply it.
+        if (half == 0 && jj > 0) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(t), (jj - 1) & 1, wc));
           if (!ok) break;
           tc_fence_after();

@@ -374,8 +374,14 @@ __global__ void __launch_bounds__(320, 1)
         }
         pk[c] = pack4_e4m3(pv[0].x, pv[0].y, pv[1].x, pv[1].y);
       }
-      // P V_{j-1} of this tile is complete (it preceded S(j) in the pipe);
-      // P goes over the first 32 columns of S, already read
+      // P goes over the first 32 columns of S (already read) once P V_{j-1},
+      // the last reader of P, is done; awaited on its own barrier, since the
+      // completion of S(j), issued after it, does not imply it
+      if (jj > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(t), (jj - 1) & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+      }
       tmem_st32(tS, pk);
       const float2 ls2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
       l += ls2.x + ls2.y;

@@ -26,7 +26,10 @@
  *    copies require; otherwise FA_ERR_ALIGNMENT.
  *  - dtype is FA_F16 or FA_BF16 for every tensor of one call; fp32 inputs
  *    are not supported (the pages' troubleshooting section: fp16/bf16 only).
- *  - head_dim d is 64 or 128.
+ *  - head_dim d is 64 or 128; the forward calls (fa_fwd, fa_fwd_varlen) also
+ *    take 256 (head dims up to 256, with the backward limited above 192:
+ *    "Что такое FlashAttention…", section on versions and hardware).  The
+ *    backward calls return FA_ERR_UNSUPPORTED for d = 256.
  *  - Hq query heads, Hkv key/value heads, Hq % Hkv == 0: query head h reads
  *    kv head h / (Hq / Hkv) (MQA/GQA, Workflow 2 Step 3).
  *  - causal != 0 hides key j from query i when j > i + (Nk - Nq) (masks are

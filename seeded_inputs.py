@@ -69,6 +69,9 @@ WORKLOADS = {
     "fwdbwd_1x16384_h16_d128_bf16_causal": Workload("fwdbwd_1x16384_h16_d128_bf16_causal", 1,
                                                     16384, 16384, 16, 16, 128, BF16, True,
                                                     seed=4, backward=True),
+    # head_dim 256, the largest the pages list, on a causal 2 x 4096 batch
+    "fwd_2x4096_h16_d256_bf16_causal": Workload("fwd_2x4096_h16_d256_bf16_causal", 2, 4096, 4096,
+                                                16, 16, 256, BF16, True, seed=9),
 }
 
 

@@ -74,7 +74,7 @@ def call_fwd(lib, q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, B=1, 
     (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
     (dict(dtype=2), fa.FA_ERR_UNSUPPORTED),
     (dict(d=96), fa.FA_ERR_UNSUPPORTED),
-    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=512), fa.FA_ERR_UNSUPPORTED),
     (dict(q=0x10008), fa.FA_ERR_ALIGNMENT),
     (dict(qs=_strides(128 * 2 * 64, 2 * 64 + 4, 64)), fa.FA_ERR_ALIGNMENT),
     (dict(o=0x10000), fa.FA_ERR_INVALID_ARG),      # output aliases q
