@@ -84,6 +84,17 @@ class Oracle:
         ipt = ctypes.POINTER(ctypes.c_int)
         lib.oracle_fwd_paged.argtypes = [dp, dp, dp, ipt, ipt, dp, dp] + [i] * 8 + [dbl, i, i, i, i]
         lib.oracle_fwd_paged.restype = i
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        u64, u32 = ctypes.c_uint64, ctypes.c_uint32
+        lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        lib.oracle_philox4x32_10.restype = i
+        lib.oracle_dropout_keep.argtypes = [u64, u32, ctypes.c_long, ctypes.c_long,
+                                            ctypes.c_long, i]
+        lib.oracle_dropout_keep.restype = i
+        lib.oracle_fwd_dropout.argtypes = [dp, dp, dp, dp, dp] + shape + [i, u64, u32, i]
+        lib.oracle_fwd_dropout.restype = i
+        lib.oracle_bwd_dropout.argtypes = [dp] * 9 + shape + [i, u64, u32, i]
+        lib.oracle_bwd_dropout.restype = i
         lib.oracle_default_threads.argtypes = []
         lib.oracle_default_threads.restype = i
         self.lib = lib
@@ -166,6 +177,50 @@ class Oracle:
             raise RuntimeError("oracle_fwd_paged failed (bad seqlen or page id?)")
         return o, lse
 
+    def philox4x32_10(self, counter, key):
+        """Philox4x32-10 of a 4-word counter and 2-word key: four uint32 words."""
+        ctr = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in counter])
+        k = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+        out = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(ctr, k, out)
+        return [int(x) for x in out]
+
+    def dropout_keep(self, seed, offset, bh, i, j, T):
+        return bool(self.lib.oracle_dropout_keep(int(seed), int(offset), int(bh), int(i), int(j),
+                                                 int(T)))
+
+    def attention_fwd_dropout(self, q, k, v, softmax_scale, keep_T, seed, offset, causal=False,
+                              window_size=(-1, -1), nthreads=0):
+        """O and LSE with dropout at keep threshold keep_T (1..255)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+        o = np.zeros((B, Nq, Hq, d), np.float64)
+        lse = np.zeros((B, Hq, Nq), np.float64)
+        c, wl, wr = _mask_args(causal, window_size)
+        rc = self.lib.oracle_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Nq, Nk,
+                                         Hq, Hkv, d, float(softmax_scale), c, wl, wr, int(keep_T),
+                                         int(seed), int(offset), int(nthreads))
+        if rc:
+            raise RuntimeError("oracle_fwd_dropout failed")
+        return o, lse
+
+    def attention_bwd_dropout(self, q, k, v, dout, softmax_scale, keep_T, seed, offset,
+                              causal=False, window_size=(-1, -1), nthreads=0):
+        """dQ, dK, dV, LSE and D with dropout at keep threshold keep_T."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        lse = np.zeros((B, Hq, Nq), np.float64)
+        D = np.zeros((B, Hq, Nq), np.float64)
+        c, wl, wr = _mask_args(causal, window_size)
+        rc = self.lib.oracle_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq),
+                                         _ptr(dk), _ptr(dv), _ptr(lse), _ptr(D), B, Nq, Nk, Hq,
+                                         Hkv, d, float(softmax_scale), c, wl, wr, int(keep_T),
+                                         int(seed), int(offset), int(nthreads))
+        if rc:
+            raise RuntimeError("oracle_bwd_dropout failed")
+        return dq, dk, dv, lse, D
+
     def attention_bwd(self, q, k, v, dout, softmax_scale, causal=False, window_size=(-1, -1),
                       nthreads=0):
         """dQ, dK, dV of L = sum(dout * O), plus the oracle's own LSE and D (fp64)."""
@@ -217,3 +272,16 @@ def attention_bwd(*a, **kw):
 
 def attention_fwd_paged(*a, **kw):
     return _get().attention_fwd_paged(*a, **kw)
+
+
+def attention_fwd_dropout(*a, **kw):
+    return _get().attention_fwd_dropout(*a, **kw)
+
+
+def attention_bwd_dropout(*a, **kw):
+    return _get().attention_bwd_dropout(*a, **kw)
+
+
+def dropout_keep_threshold(p: float) -> int:
+    """T = round(256 (1 - p)): an element is kept iff its random byte is below T."""
+    return int(round(256.0 * (1.0 - float(p))))

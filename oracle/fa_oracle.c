@@ -32,6 +32,15 @@
  *   - GQA maps query head h to kv head h / (Hq / Hkv) (consecutive groups);
  *   - LSE is the natural log of sum_j exp(S_ij) over visible keys;
  *   - a row with no visible key has O = 0, LSE = -inf, and zero gradients;
+ *   - dropout (optional) multiplies P_ij by s M_ij before P V, where M_ij is
+ *     a keep bit and s = 256 / T the rescale, and leaves LSE alone; M_ij is
+ *     read from Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel
+ *     random numbers: as easy as 1, 2, 3", SC 2011) with key = the 64-bit seed
+ *     and counter (j / 4, i / 4, b Hq + h, offset): the byte (j mod 4) of
+ *     output word (i mod 4) keeps the element iff it is below T = round(256
+ *     (1 - p)) ("optimizing-attention-flash", the dropout_p argument of
+ *     flash_attn_func; "Что такое FlashAttention…", versions section: dropout
+ *     among the features);
  *   - backward is the textbook gradient of the definition:
  *       dV = P^T dO, dP = dO V^T, D_i = sum_j P_ij dP_ij,
  *       dS = P o (dP - D), dQ = tau dS K, dK = tau dS^T Q
@@ -54,7 +63,54 @@ typedef struct {
     int B, Nq, Nk, Hq, Hkv, d;
     double tau;
     int causal, wl, wr;
+    /* dropout: keep threshold T in [1, 255] (0 = no dropout), Philox key and
+     * counter offset */
+    int drop_T;
+    uint64_t drop_seed;
+    uint32_t drop_offset;
 } shape_t;
+
+/* Philox4x32-10 (SC 2011): ten rounds of two 32 x 32 -> 64-bit products
+ * with multipliers 0xD2511F53 and 0xCD9E8D57; between rounds the key is
+ * bumped by the Weyl constants 0x9E3779B9 and 0xBB67AE85. */
+int oracle_philox4x32_10(const uint32_t* ctr, const uint32_t* key, uint32_t* out) {
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * x0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * x2;
+        uint32_t y0 = (uint32_t)(p1 >> 32) ^ x1 ^ k0;
+        uint32_t y1 = (uint32_t)p1;
+        uint32_t y2 = (uint32_t)(p0 >> 32) ^ x3 ^ k1;
+        uint32_t y3 = (uint32_t)p0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+    return 0;
+}
+
+/* Keep bit of element (i, j) of (batch, query head) bh: 1 or 0. */
+int oracle_dropout_keep(uint64_t seed, uint32_t offset, long bh, long i, long j, int T) {
+    uint32_t ctr[4] = {(uint32_t)(j / 4), (uint32_t)(i / 4), (uint32_t)bh, offset};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    oracle_philox4x32_10(ctr, key, w);
+    uint32_t byte = (w[i % 4] >> (8 * (j % 4))) & 0xFFu;
+    return byte < (uint32_t)T;
+}
+
+/* Multiplier of P_ij in P V: s M_ij with dropout, 1 without. */
+static double drop_mult(const shape_t* s, int b, int h, long i, long j) {
+    if (s->drop_T <= 0) return 1.0;
+    long bh = (long)b * s->Hq + h;
+    return oracle_dropout_keep(s->drop_seed, s->drop_offset, bh, i, j, s->drop_T)
+               ? 256.0 / s->drop_T
+               : 0.0;
+}
 
 /* Is key j visible to query i?  (mask definition, see header) */
 static int key_visible(const shape_t* s, long i, long j) {
@@ -187,7 +243,8 @@ static void fwd_one_row(const fwd_ctx* c, int b, int h, int i, double* out_o, do
     for (int j = 0; j < s->Nk; ++j) {
         if (prow[j] == 0.0) continue;
         const double* vj = kv_row(c->v, s, b, j, g);
-        for (int cc = 0; cc < s->d; ++cc) out_o[cc] += prow[j] * vj[cc];
+        double zij = prow[j] * drop_mult(s, b, h, i, j);
+        for (int cc = 0; cc < s->d; ++cc) out_o[cc] += zij * vj[cc];
     }
     *out_lse = lse;
 }
@@ -360,7 +417,8 @@ static void bwd_row_item(void* ctx, long item, double* scratch) {
     const double* doi = c->dout + (((size_t)b * s->Nq + i) * s->Hq + h) * s->d;
     double Di = 0.0;
     for (int j = 0; j < s->Nk; ++j) {
-        dprow[j] = dot(doi, kv_row(c->v, s, b, j, g), s->d);
+        /* gradient w.r.t. P_ij: dO_i . V_j through the dropout multiplier */
+        dprow[j] = dot(doi, kv_row(c->v, s, b, j, g), s->d) * drop_mult(s, b, h, i, j);
         Di += prow[j] * dprow[j];
     }
     double* dqi = c->dq + (((size_t)b * s->Nq + i) * s->Hq + h) * s->d;
@@ -401,11 +459,13 @@ static void bwd_key_item(void* ctx, long item, double* scratch) {
             const double* doi = c->dout + (((size_t)b * s->Nq + i) * s->Hq + h) * s->d;
             double Sij = s->tau * dot(qi, kj, s->d);
             double Pij = exp(Sij - lse);
-            double dPij = dot(doi, vj, s->d);
+            double mult = drop_mult(s, b, h, i, j);
+            double Zij = Pij * mult; /* the weight of V_j in O_i */
+            double dPij = dot(doi, vj, s->d) * mult;
             double dSij = Pij * (dPij - c->Dvec[li]);
             for (int cc = 0; cc < s->d; ++cc) {
                 dkj[cc] += s->tau * dSij * qi[cc];
-                dvj[cc] += Pij * doi[cc];
+                dvj[cc] += Zij * doi[cc];
             }
         }
     }
@@ -418,6 +478,40 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
                int Hq, int Hkv, int d, double tau, int causal, int window_left, int window_right,
                int nthreads) {
     bwd_ctx c = {{B, Nq, Nk, Hq, Hkv, d, tau, causal, window_left, window_right},
+                 q, k, v, dout, dq, dk, dv, NULL, NULL};
+    if (check_shape(&c.s)) return -1;
+    size_t nrow = (size_t)B * Hq * Nq;
+    c.lse = lse_out ? lse_out : (double*)malloc(sizeof(double) * nrow);
+    c.Dvec = D_out ? D_out : (double*)malloc(sizeof(double) * nrow);
+    int rc = -1;
+    if (c.lse && c.Dvec) {
+        rc = run_pool(bwd_row_item, &c, (long)nrow, 3 * (size_t)Nk, nthreads);
+        if (rc == 0) rc = run_pool(bwd_key_item, &c, (long)B * Hkv * Nk, 1, nthreads);
+    }
+    if (!lse_out) free(c.lse);
+    if (!D_out) free(c.Dvec);
+    return rc;
+}
+
+/* The forward and backward with dropout at keep threshold T (1..255). */
+int oracle_fwd_dropout(const double* q, const double* k, const double* v, double* o, double* lse,
+                       int B, int Nq, int Nk, int Hq, int Hkv, int d, double tau, int causal,
+                       int window_left, int window_right, int T, uint64_t seed, uint32_t offset,
+                       int nthreads) {
+    if (T < 1 || T > 255) return -1;
+    fwd_ctx c = {{B, Nq, Nk, Hq, Hkv, d, tau, causal, window_left, window_right, T, seed, offset},
+                 q, k, v, o, lse, NULL};
+    if (check_shape(&c.s)) return -1;
+    return run_pool(fwd_item, &c, (long)B * Hq * Nq, 2 * (size_t)Nk, nthreads);
+}
+
+int oracle_bwd_dropout(const double* q, const double* k, const double* v, const double* dout,
+                       double* dq, double* dk, double* dv, double* lse_out, double* D_out, int B,
+                       int Nq, int Nk, int Hq, int Hkv, int d, double tau, int causal,
+                       int window_left, int window_right, int T, uint64_t seed, uint32_t offset,
+                       int nthreads) {
+    if (T < 1 || T > 255) return -1;
+    bwd_ctx c = {{B, Nq, Nk, Hq, Hkv, d, tau, causal, window_left, window_right, T, seed, offset},
                  q, k, v, dout, dq, dk, dv, NULL, NULL};
     if (check_shape(&c.s)) return -1;
     size_t nrow = (size_t)B * Hq * Nq;

@@ -14,6 +14,9 @@ Each check below ties the oracle to a source independent of its code:
     and folded into the output with correct normalisation, must equal full
     attention;
   * central finite differences and fp64 torch autograd for the backward;
+  * for dropout, the generator's published known-answer vectors, a brute
+    force whose mask is decoded in Python from the generator's words, the
+    keep rate, and central finite differences of the dropout forward;
   * for the paged KV cache, equality with the (pinned) contiguous definition
     on the gathered keys, through a permuted page table with unrelated
     values in every row and page the sequence does not own.
@@ -399,9 +402,82 @@ def check_paged(orc):
         np.testing.assert_allclose(lse[b:b + 1], lseb, rtol=0, atol=1e-12)
 
 
+def check_philox_kat(orc):
+    # the generator behind dropout against its authors' known-answer vectors
+    with open(os.path.join(GOLDEN, "philox4x32_10_kat.json")) as f:
+        kat = json.load(f)
+    for vec in kat["vectors"]:
+        ctr = [int(x, 16) for x in vec["counter"]]
+        key = [int(x, 16) for x in vec["key"]]
+        assert orc.philox4x32_10(ctr, key) == [int(x, 16) for x in vec["out"]]
+
+
+def dropout_mask_bruteforce(orc, seed, offset, B, Hq, Nq, Nk, T):
+    """Keep mask [B, Hq, Nq, Nk] decoded here from the (KAT-pinned) generator:
+    counter (j // 4, i // 4, b Hq + h, offset), key = seed split in two words,
+    byte j % 4 of word i % 4, kept iff below T."""
+    m = np.zeros((B, Hq, Nq, Nk), bool)
+    key = [seed & 0xFFFFFFFF, seed >> 32]
+    for b in range(B):
+        for h in range(Hq):
+            for ib in range(0, Nq, 4):
+                for jb in range(0, Nk, 4):
+                    w = orc.philox4x32_10([jb // 4, ib // 4, b * Hq + h, offset], key)
+                    for i in range(ib, min(ib + 4, Nq)):
+                        for j in range(jb, min(jb + 4, Nk)):
+                            m[b, h, i, j] = ((w[i % 4] >> (8 * (j % 4))) & 0xFF) < T
+    return m
+
+
+def check_dropout(orc):
+    seed, offset = 0x1234567890ABCDEF, 3
+    for (causal, window), (Hq, Hkv), T in itertools.product(
+            [(False, (-1, -1)), (True, (-1, -1)), (False, (2, 1))], [(4, 2)], [26, 179]):
+        B, Nq, Nk, d = 2, 7, 9, 3
+        q, k, v = rand((B, Nq, Hq, d), 151), rand((B, Nk, Hkv, d), 152), rand((B, Nk, Hkv, d), 153)
+        o, lse = orc.attention_fwd_dropout(q, k, v, 0.7, T, seed, offset, causal, window)
+        # brute force: the plain probabilities (pinned above), the mask decoded
+        # here, and O = (256 / T) sum_j P_ij M_ij V_j; LSE is the plain one
+        m = dropout_mask_bruteforce(orc, seed, offset, B, Hq, Nq, Nk, T)
+        G = Hq // Hkv
+        ob = np.zeros_like(o)
+        for b in range(B):
+            for h in range(Hq):
+                P = orc.attention_probs(q, k, b, h, 0.7, causal, window)
+                Z = P * m[b, h] * (256.0 / T)
+                ob[b, :, h, :] = Z @ v[b, :, h // G, :]
+        np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+        _, lse_plain = orc.attention_fwd(q, k, v, 0.7, causal, window)
+        np.testing.assert_array_equal(lse, lse_plain)
+    # the keep rate over many elements is T / 256 (binomial, 5 sigma)
+    m = dropout_mask_bruteforce(orc, 77, 0, 1, 2, 64, 64, 64)
+    n, kept = m.size, m.sum()
+    assert abs(kept - n * 0.25) <= 5 * math.sqrt(n * 0.25 * 0.75)
+    # the backward is the gradient of the dropout forward (fixed mask): central
+    # finite differences of L = sum(dout * O)
+    B, Nq, Nk, Hq, Hkv, d, T = 1, 5, 6, 2, 1, 3, 128
+    q, k, v = rand((B, Nq, Hq, d), 161), rand((B, Nk, Hkv, d), 162), rand((B, Nk, Hkv, d), 163)
+    do = rand((B, Nq, Hq, d), 164)
+    dq, dk, dv, _, _ = orc.attention_bwd_dropout(q, k, v, do, 0.6, T, 9, 1, True)
+
+    def loss(qq, kk, vv):
+        return float((orc.attention_fwd_dropout(qq, kk, vv, 0.6, T, 9, 1, True)[0] * do).sum())
+    eps = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if y is x else y for y in (q, k, v)]
+            args_m = [xm if y is x else y for y in (q, k, v)]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
 ALL_CHECKS = [check_bruteforce, check_library_fwd, check_golden, check_closed_forms,
               check_invariants, check_mqa_equivalence, check_walkthrough, check_backward,
-              check_empty_rows, check_paged]
+              check_empty_rows, check_paged, check_philox_kat, check_dropout]
 
 
 @pytest.fixture(scope="module")
@@ -465,7 +541,7 @@ MUTATIONS = {
                         "double dS = prow[j] * (Di - dprow[j]);"),
     "D dropped in dK": ("double dSij = Pij * (dPij - c->Dvec[li]);", "double dSij = Pij * dPij;"),
     "dK without scale": ("dkj[cc] += s->tau * dSij * qi[cc];", "dkj[cc] += dSij * qi[cc];"),
-    "dV uses dS": ("dvj[cc] += Pij * doi[cc];", "dvj[cc] += dSij * doi[cc];"),
+    "dV uses dS": ("dvj[cc] += Zij * doi[cc];", "dvj[cc] += dSij * doi[cc];"),
     "dQ uses V": ("const double* kj = kv_row(c->k, s, b, j, g);\n        for",
                   "const double* kj = kv_row(c->v, s, b, j, g);\n        for"),
     "one head per kv group in dK": ("for (int h = g * G; h < (g + 1) * G; ++h)",
@@ -475,6 +551,14 @@ MUTATIONS = {
                                "int nk = c->seqlens[b] > 0 ? c->seqlens[b] - 1 : 0;"),
     "paged mask aligned top-left": ("shape_t s = {1, c->Nq, nk,", "shape_t s = {1, c->Nq, c->Nq,"),
     "paged kv head interleaved": ("int kv_head = h / (c->Hq / c->Hkv);", "int kv_head = h % c->Hkv;"),
+    "philox key bump skipped": ("k0 += 0x9E3779B9u;", ""),
+    "dropout byte from the wrong word": ("uint32_t byte = (w[i % 4] >> (8 * (j % 4))) & 0xFFu;",
+                                         "uint32_t byte = (w[j % 4] >> (8 * (i % 4))) & 0xFFu;"),
+    "dropout rescale missing": ("? 256.0 / s->drop_T", "? 1.0"),
+    "dropout mask left out of dP": (
+        "dprow[j] = dot(doi, kv_row(c->v, s, b, j, g), s->d) * drop_mult(s, b, h, i, j);",
+        "dprow[j] = dot(doi, kv_row(c->v, s, b, j, g), s->d);"),
+    "dV without the dropout mask": ("double Zij = Pij * mult;", "double Zij = Pij;"),
 }
 
 
