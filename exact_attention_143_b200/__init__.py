@@ -37,7 +37,8 @@ FA_ERR_DEVICE_TIMEOUT = 6
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
             "fa_bwd_noalloc", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
-            "fa_fwd_paged_workspace_size", "fa_fwd_paged", "fa_fwd_fp8")
+            "fa_fwd_paged_workspace_size", "fa_fwd_paged", "fa_fwd_fp8", "fa_fwd_dropout",
+            "fa_bwd_dropout")
 
 _lib = None
 
@@ -90,6 +91,13 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_paged.restype = i
     lib.fa_fwd_fp8.argtypes = [vp] * 5 + [i] * 6 + [i64p] * 4 + [f] * 4 + [i, i, i, vp]
     lib.fa_fwd_fp8.restype = i
+    u64, u32 = ctypes.c_uint64, ctypes.c_uint32
+    lib.fa_fwd_dropout.argtypes = ([vp, vp, vp, vp, vp, i, i, i, i, i, i, i64p, i64p, i64p, i64p,
+                                    i, f, i, i, i, f, u64, u32, vp])
+    lib.fa_fwd_dropout.restype = i
+    lib.fa_bwd_dropout.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [i] * 6 + [i64p] * 8 +
+                                   [i, f, i, i, i, f, u64, u32, vp])
+    lib.fa_bwd_dropout.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -134,8 +142,14 @@ def _stream(dev):
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
-def fa_fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), out=None, lse=None):
-    """Exact attention forward; returns (o [B,Nq,Hq,d], lse [B,Hq,Nq] fp32)."""
+def fa_fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), out=None, lse=None,
+           dropout_p=0.0, seed=0, offset=0):
+    """Exact attention forward; returns (o [B,Nq,Hq,d], lse [B,Hq,Nq] fp32).
+
+    With dropout_p > 0 the probabilities are dropped before P V (keep bits
+    from Philox4x32-10 keyed by `seed`, counter offset `offset`; the kept ones
+    are rescaled by 256 / round(256 (1 - dropout_p))); pass the same seed and
+    offset to fa_bwd."""
     lib = load_library()
     dev = _check_cuda(q, k, v)
     code = _dtype_code(q)
@@ -152,10 +166,17 @@ def fa_fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), out=
         raise ValueError("lse must be a contiguous fp32 [B, Hq, Nq] tensor")
     wl, wr = window_size
     with torch.cuda.device(dev):
-        rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                        B, Nq, Nk, Hq, Hkv, d, _strides(q), _strides(k), _strides(v),
-                        _strides(out), code, _scale(softmax_scale, d), int(bool(causal)),
-                        int(wl), int(wr), _stream(dev))
+        if dropout_p:
+            rc = lib.fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, Nq, Nk, Hq, Hkv, d, _strides(q),
+                                    _strides(k), _strides(v), _strides(out), code,
+                                    _scale(softmax_scale, d), int(bool(causal)), int(wl), int(wr),
+                                    float(dropout_p), int(seed), int(offset), _stream(dev))
+        else:
+            rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            lse.data_ptr(), B, Nq, Nk, Hq, Hkv, d, _strides(q), _strides(k),
+                            _strides(v), _strides(out), code, _scale(softmax_scale, d),
+                            int(bool(causal)), int(wl), int(wr), _stream(dev))
     if rc:
         raise FAError(rc, "fa_fwd")
     return out, lse
@@ -254,7 +275,7 @@ def bwd_workspace_size(B, Nq, Hq, d) -> int:
 
 
 def fa_bwd(dout, q, k, v, o, lse, softmax_scale=None, causal=False, window_size=(-1, -1),
-           dq=None, dk=None, dv=None, workspace=None):
+           dq=None, dk=None, dv=None, workspace=None, dropout_p=0.0, seed=0, offset=0):
     """Exact attention backward from the forward's O and LSE; returns (dq, dk, dv)."""
     lib = load_library()
     dev = _check_cuda(dout, q, k, v, o, lse)
@@ -274,14 +295,16 @@ def fa_bwd(dout, q, k, v, o, lse, softmax_scale=None, causal=False, window_size=
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     _check_cuda(q, dq, dk, dv, workspace)
     wl, wr = window_size
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), B, Nq, Nk, Hq, Hkv, d, _strides(q),
+            _strides(k), _strides(v), _strides(o), _strides(dout), _strides(dq), _strides(dk),
+            _strides(dv), code, _scale(softmax_scale, d), int(bool(causal)), int(wl), int(wr))
     with torch.cuda.device(dev):
-        rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
-                        lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                        B, Nq, Nk, Hq, Hkv, d, _strides(q), _strides(k), _strides(v),
-                        _strides(o), _strides(dout), _strides(dq), _strides(dk), _strides(dv),
-                        code, _scale(softmax_scale, d), int(bool(causal)), int(wl), int(wr),
-                        _stream(dev))
+        if dropout_p:
+            rc = lib.fa_bwd_dropout(*args, float(dropout_p), int(seed), int(offset), _stream(dev))
+        else:
+            rc = lib.fa_bwd(*args, _stream(dev))
     if rc:
         raise FAError(rc, "fa_bwd")
     return dq, dk, dv

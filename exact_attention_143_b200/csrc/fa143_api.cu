@@ -158,11 +158,11 @@ __global__ void fa_selftest_wait_kernel(unsigned int* err, uint64_t limit_ns) {
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const fa::FwdParams& prm, cudaStream_t st) {
   using Cfg = fa::FwdCfg<D>;
-  auto kern = fa::fa_fwd_kernel<D, BF16>;
+  auto kern = fa::fa_fwd_kernel<D, BF16, DROP>;
   static bool attr_done = false;  // per instantiation and process
   if (!attr_done) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -208,14 +208,14 @@ int make_dq_acc_map(CUtensorMap* map, float* dq_acc, int B, int Nq, int Hq, int 
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP = false>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mdo, const fa::BwdParams& prm, cudaStream_t st) {
   CUtensorMap mdq;
   int rc = make_dq_acc_map(&mdq, prm.dq_acc, prm.B, prm.Nq, prm.Hq, D, 128);
   if (rc) return rc;
   using Cfg = fa::BwdCfg<D>;
-  auto kern = fa::fa_bwd_main_kernel<D, BF16>;
+  auto kern = fa::fa_bwd_main_kernel<D, BF16, DROP>;
   static bool attr_done = false;  // per instantiation and process
   if (!attr_done) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -281,7 +281,7 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
              const TensorDesc& to, float* lse, size_t lse_bytes, int B, int Nq, int Nk, int Hq,
              int Hkv, int d, const int* cu_q, const int* cu_k, int total_q, int total_k,
              int dtype, float softmax_scale, int causal, int window_left, int window_right,
-             void* stream) {
+             void* stream, const fa::DropoutParams* drop = nullptr) {
   int rc;
   for (const TensorDesc* t : {&tq, &tk, &tv, &to})
     if ((rc = check_tensor(*t))) return rc;
@@ -320,8 +320,17 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   prm.cu_k = cu_k;
   prm.total_q = total_q;
   prm.total_k = total_k;
+  if (drop) prm.drop = *drop;
   if (!prm.err) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (drop) {
+    if (d == 256 || cu_q) return FA_ERR_UNSUPPORTED;
+    if (dtype == FA_BF16)
+      return d == 64 ? launch_fwd<64, true, true>(mq, mk, mv, prm, st)
+                     : launch_fwd<128, true, true>(mq, mk, mv, prm, st);
+    return d == 64 ? launch_fwd<64, false, true>(mq, mk, mv, prm, st)
+                   : launch_fwd<128, false, true>(mq, mk, mv, prm, st);
+  }
   if (d == 256)
     return dtype == FA_BF16 ? launch_fwd256<true>(mq, mk, mv, prm, st)
                             : launch_fwd256<false>(mq, mk, mv, prm, st);
@@ -403,8 +412,10 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
              const TensorDesc& tdk, const TensorDesc& tdv, const float* lse, size_t lse_bytes,
              void* workspace, size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv,
              int d, const int* cu_q, const int* cu_k, int total_q, int total_k, int dtype,
-             float softmax_scale, int causal, int window_left, int window_right, void* stream) {
+             float softmax_scale, int causal, int window_left, int window_right, void* stream,
+             const fa::DropoutParams* drop = nullptr) {
   int rc;
+  if (drop && cu_q) return FA_ERR_UNSUPPORTED;
   for (const TensorDesc* t : {&tq, &tk, &tv, &to, &tdo, &tdq, &tdk, &tdv})
     if ((rc = check_tensor(*t))) return rc;
   if (!lse) return FA_ERR_INVALID_ARG;
@@ -505,13 +516,22 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   bp.cu_k = cu_k;
   bp.total_q = total_q;
   bp.total_k = total_k;
+  if (drop) bp.drop = *drop;
   if (g_bwd_ev_start && cudaEventRecord(g_bwd_ev_start, st) != cudaSuccess) return FA_ERR_CUDA;
-  if (bf16)
+  if (drop) {
+    if (bf16)
+      rc = d == 64 ? launch_bwd<64, true, true>(mq, mk, mv, mdo, bp, st)
+                   : launch_bwd<128, true, true>(mq, mk, mv, mdo, bp, st);
+    else
+      rc = d == 64 ? launch_bwd<64, false, true>(mq, mk, mv, mdo, bp, st)
+                   : launch_bwd<128, false, true>(mq, mk, mv, mdo, bp, st);
+  } else if (bf16) {
     rc = d == 64 ? launch_bwd<64, true>(mq, mk, mv, mdo, bp, st)
                  : launch_bwd<128, true>(mq, mk, mv, mdo, bp, st);
-  else
+  } else {
     rc = d == 64 ? launch_bwd<64, false>(mq, mk, mv, mdo, bp, st)
                  : launch_bwd<128, false>(mq, mk, mv, mdo, bp, st);
+  }
   if (rc) return rc;
   if (g_bwd_ev_stop && cudaEventRecord(g_bwd_ev_stop, st) != cudaSuccess) return FA_ERR_CUDA;
 
@@ -1023,6 +1043,96 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_fwd_fp8<64>(mq, mk, mv, prm, st)
                  : launch_fwd_fp8<128>(mq, mk, mv, prm, st);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ dropout
+namespace {
+
+// Keep threshold of dropout probability p: T = round(256 (1 - p)).  Returns
+// FA_OK with *T in [1, 256] (256: nothing is dropped), or INVALID_ARG.
+int dropout_threshold(float p, int* T) {
+  if (!std::isfinite(p) || p < 0.f || p >= 1.f) return FA_ERR_INVALID_ARG;
+  const int t = int(std::lround(256.0 * (1.0 - double(p))));
+  if (t < 1) return FA_ERR_INVALID_ARG;
+  *T = std::min(t, 256);
+  return FA_OK;
+}
+
+fa::DropoutParams make_dropout(int T, uint64_t seed, uint32_t offset) {
+  fa::DropoutParams dp{};
+  dp.T = uint32_t(T);
+  dp.seed_lo = uint32_t(seed);
+  dp.seed_hi = uint32_t(seed >> 32);
+  dp.offset = offset;
+  dp.scale = 256.f / float(T);
+  return dp;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int Nq, int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3],
+                   const int64_t k_stride[3], const int64_t v_stride[3],
+                   const int64_t o_stride[3], int dtype, float softmax_scale, int causal,
+                   int window_left, int window_right, float dropout_p, uint64_t seed,
+                   uint32_t offset, void* stream) {
+  int T = 0;
+  int rc = dropout_threshold(dropout_p, &T);
+  if (rc) return rc;
+  if (T >= 256)  // nothing is dropped
+    return fa_fwd(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride,
+                  dtype, softmax_scale, causal, window_left, window_right, stream);
+  rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  if (rc) return rc;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  const fa::DropoutParams dp = make_dropout(T, seed, offset);
+  return fwd_impl(tq, tk, tv, to, lse, size_t(B) * Hq * Nq * sizeof(float), B, Nq, Nk, Hq, Hkv,
+                  d, nullptr, nullptr, 0, 0, dtype, softmax_scale, causal, window_left,
+                  window_right, stream, &dp);
+}
+
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                   const int64_t q_stride[3], const int64_t k_stride[3],
+                   const int64_t v_stride[3], const int64_t o_stride[3],
+                   const int64_t do_stride[3], const int64_t dq_stride[3],
+                   const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
+                   float softmax_scale, int causal, int window_left, int window_right,
+                   float dropout_p, uint64_t seed, uint32_t offset, void* stream) {
+  int T = 0;
+  int rc = dropout_threshold(dropout_p, &T);
+  if (rc) return rc;
+  if (T >= 256)
+    return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Nq, Nk, Hq,
+                  Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride,
+                  dk_stride, dv_stride, dtype, softmax_scale, causal, window_left, window_right,
+                  stream);
+  rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  if (rc) return rc;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
+      !dk_stride || !dv_stride)
+    return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
+  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
+  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdo{dout, do_stride[0], do_stride[1], do_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdq{dq, dq_stride[0], dq_stride[1], dq_stride[2], B, Nq, Hq, d};
+  const TensorDesc tdk{dk, dk_stride[0], dk_stride[1], dk_stride[2], B, Nk, Hkv, d};
+  const TensorDesc tdv{dv, dv_stride[0], dv_stride[1], dv_stride[2], B, Nk, Hkv, d};
+  const fa::DropoutParams dp = make_dropout(T, seed, offset);
+  return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(B) * Hq * Nq * sizeof(float),
+                  workspace, workspace_bytes, B, Nq, Nk, Hq, Hkv, d, nullptr, nullptr, 0, 0,
+                  dtype, softmax_scale, causal, window_left, window_right, stream, &dp);
 }
 
 }  // extern "C"

@@ -52,6 +52,7 @@
 #include <cuda_fp16.h>
 
 #include "fa_ptx.cuh"
+#include "fa_dropout.cuh"
 #include "fa_exp2.cuh"
 
 namespace fa {
@@ -190,6 +191,7 @@ struct BwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  DropoutParams drop;  // used by the DROP instantiations only
 };
 
 template <int D>
@@ -230,7 +232,7 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
       : "memory");
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -600,13 +602,27 @@ __global__ void __launch_bounds__(512, 1)
       if (!(ok = wait_all(bar_s, s & 1))) break;
       tc_fence_after();
       // P^T = exp2(S^T * scale * log2 e - LSE2), 32 queries at a time; a share
-      // of the query pairs takes the FMA-pipe exp2
+      // of the query pairs takes the FMA-pipe exp2.  With dropout the dV
+      // operand Z^T = P^T o M^T goes to [colP, colP + 32) and the undropped
+      // P^T, which dS needs, to [colP + 32, colP + 64) until dS^T replaces it;
+      // all of S^T is read first since those columns still hold it.
+      uint32_t srall[DROP ? 64 : 1];
+      uint32_t kwd[DROP ? 16 : 1];
+      if constexpr (DROP) {
+        tmem_ld32(Ra + colS, *reinterpret_cast<uint32_t(*)[32]>(&srall[0]));
+        tmem_ld32(Ra + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&srall[32]));
+        tmem_wait_ld();
+        dropout_col_words(p.drop, uint32_t(b * p.Hq + step_head(s)), key, q0, kwd);
+      }
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t sr[32];
-        tmem_ld32(Ra + colS + c0, sr);
-        tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t sr_own[DROP ? 1 : 32];
+        const uint32_t* sr = DROP ? &srall[c0] : sr_own;
+        if constexpr (!DROP) {
+          tmem_ld32(Ra + colS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr_own[0]));
+          tmem_wait_ld();
+        }
+        uint32_t pk[16], zk[DROP ? 16 : 1];
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
@@ -636,9 +652,20 @@ __global__ void __launch_bounds__(512, 1)
           }
           pk[c / 2] = pack2<BF16>(pv[0], pv[1]);
           pk[c / 2 + 1] = pack2<BF16>(pv[2], pv[3]);
+          if constexpr (DROP) {  // queries c0 + c .. + 3 form one group of four
+            const uint32_t wd = kwd[(c0 + c) >> 2];
+            zk[c / 2] = pack2<BF16>(pv[0] * keep_of(wd, 0, p.drop.T), pv[1] * keep_of(wd, 1, p.drop.T));
+            zk[c / 2 + 1] =
+                pack2<BF16>(pv[2] * keep_of(wd, 2, p.drop.T), pv[3] * keep_of(wd, 3, p.drop.T));
+          }
         }
-        // packed P^T written over S^T columns this thread has already read
-        tmem_st16(Ra + colP + c0 / 2, pk);
+        if constexpr (DROP) {
+          tmem_st16(Ra + colP + c0 / 2, zk);
+          tmem_st16(Ra + colP + 32 + c0 / 2, pk);
+        } else {
+          // packed P^T written over S^T columns this thread has already read
+          tmem_st16(Ra + colP + c0 / 2, pk);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -650,17 +677,32 @@ __global__ void __launch_bounds__(512, 1)
       if (!(ok = wait_all(bar_dp, s & 1))) break;
       tc_fence_after();
       uint8_t* dsrow = smem + Cfg::kSmemDS + half * Cfg::kChunk + j * 128;
-      uint32_t dpr[64];
-      tmem_ld32(Rb + colS, *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]));
-      tmem_ld32(Rb + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_dpfree);
+      uint32_t dpr[DROP ? 32 : 64];
+      if constexpr (!DROP) {
+        tmem_ld32(Rb + colS, *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]));
+        tmem_ld32(Rb + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_dpfree);
+      }
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t pr[16], dk[16];
-        tmem_ld16(Ra + colP + c0 / 2, pr);
-        tmem_wait_ld();
+        uint32_t pr[16], dk[16], zr[DROP ? 16 : 1];
+        const uint32_t* dpc = DROP ? dpr : &dpr[c0 % (DROP ? 32 : 64)];
+        if constexpr (DROP) {
+          // dP^T chunk, Z^T (whose zeros are the dropped pairs) and P^T
+          tmem_ld32(Rb + colS + c0, *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]));
+          tmem_ld16(Ra + colP + c0 / 2, *reinterpret_cast<uint32_t(*)[16]>(&zr[0]));
+          tmem_ld16(Ra + colP + 32 + c0 / 2, pr);
+          tmem_wait_ld();
+          if (c0 == 32) {  // all of dP^T(s) is in registers
+            tc_fence_before();
+            mbar_arrive(bar_dpfree);
+          }
+        } else {
+          tmem_ld16(Ra + colP + c0 / 2, pr);
+          tmem_wait_ld();
+        }
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const float4 d4 = *reinterpret_cast<const float4*>(Dv + c0 + c);
@@ -679,18 +721,26 @@ __global__ void __launch_bounds__(512, 1)
             pf[2] = bb.x;
             pf[3] = bb.y;
           }
+          float dq4[4] = {__uint_as_float(dpc[c]), __uint_as_float(dpc[c + 1]),
+                          __uint_as_float(dpc[c + 2]), __uint_as_float(dpc[c + 3])};
+          if constexpr (DROP) {  // dP through the dropout multiplier
+            const uint32_t za = zr[c / 2], zb = zr[c / 2 + 1];
+            dq4[0] = (za & 0xFFFFu) ? dq4[0] * p.drop.scale : 0.f;
+            dq4[1] = (za >> 16) ? dq4[1] * p.drop.scale : 0.f;
+            dq4[2] = (zb & 0xFFFFu) ? dq4[2] * p.drop.scale : 0.f;
+            dq4[3] = (zb >> 16) ? dq4[3] * p.drop.scale : 0.f;
+          }
           const float2 d01 = __fmul2_rn(make_float2(pf[0], pf[1]),
-                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c0 + c]),
-                                                               __uint_as_float(dpr[c0 + c + 1])),
+                                        __fadd2_rn(make_float2(dq4[0], dq4[1]),
                                                    make_float2(-d4.x, -d4.y)));
           const float2 d23 = __fmul2_rn(make_float2(pf[2], pf[3]),
-                                        __fadd2_rn(make_float2(__uint_as_float(dpr[c0 + c + 2]),
-                                                               __uint_as_float(dpr[c0 + c + 3])),
+                                        __fadd2_rn(make_float2(dq4[2], dq4[3]),
                                                    make_float2(-d4.z, -d4.w)));
           dk[c / 2] = pack2<BF16>(d01.x, d01.y);
           dk[c / 2 + 1] = pack2<BF16>(d23.x, d23.y);
         }
-        // columns of S^T(s) this thread has already read
+        // columns of S^T(s) this thread has already read (with dropout: the
+        // P^T chunk just loaded)
         tmem_st16(Ra + colP + 32 + c0 / 2, dk);
         // smem copy in the MN-major 128-byte-swizzled layout of the dQ A operand:
         // chunk `half` holds queries [64 half, 64 half + 64) of every key row;
@@ -721,7 +771,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = (which == 0 ? Cfg::kColDK : Cfg::kColDV) + half * (D / 2);
-        const float mul = which == 0 ? p.scale : 1.f;
+        const float mul = which == 0 ? p.scale : (DROP ? p.drop.scale : 1.f);
         uint16_t* dst_row = which == 0 ? dkrow : dvrow;
 #pragma unroll
         for (int c0 = 0; c0 < D / 2; c0 += 32) {

@@ -32,6 +32,7 @@
 // a tile can see are skipped whole.
 #pragma once
 
+#include "fa_dropout.cuh"
 #include "fa_exp2.cuh"
 #include "fa_ptx.cuh"
 
@@ -55,6 +56,7 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  DropoutParams drop;  // used by the DROP instantiations only
 };
 
 template <int D>
@@ -97,7 +99,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP = false>
 __global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -475,6 +477,9 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
+        uint32_t kw[16];  // dropout keep bytes of this row for the half's 64 keys
+        if constexpr (DROP)
+          dropout_row_words(p.drop, uint32_t(b * p.Hq + h), row, key0 + 64 * half, kw);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int cc = 32 * half + c;  // column pair
@@ -487,6 +492,10 @@ __global__ void __launch_bounds__(352, 1)
             pv.y = fast_exp2(x.y);
           }
           lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);
+          if constexpr (DROP) {  // l keeps the undropped sum
+            pv.x *= keep_of(kw[c >> 1], (c & 1) * 2, p.drop.T);
+            pv.y *= keep_of(kw[c >> 1], (c & 1) * 2 + 1, p.drop.T);
+          }
           pk[c] = pack2<BF16>(pv.x, pv.y);
         }
         // P_t V_{j-1}, the last reader of P_t, must be complete before P_t is
@@ -527,7 +536,7 @@ __global__ void __launch_bounds__(352, 1)
     if (ok) {
       tc_fence_after();
       const bool has = (n > 0) && (l > 0.f);
-      const float inv_l = has ? 1.f / l : 0.f;
+      const float inv_l = has ? (DROP ? p.drop.scale : 1.f) / l : 0.f;
       const float lse = has ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const bool store = row < Nq;
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + bc * p.o_sb + int64_t(qstart + row) * p.o_ss +

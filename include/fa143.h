@@ -123,6 +123,35 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                   int window_right, void* stream);
 
 /*
+ * Forward and backward with dropout on the attention probabilities
+ * ("optimizing-attention-flash", the dropout_p argument of flash_attn_func).
+ * P_ij is multiplied by (256 / T) M_ij before P V, T = round(256 (1 - p)),
+ * where the keep bit M_ij of element (i, j) of (batch b, query head h) is
+ * byte (j mod 4) of output word (i mod 4) of Philox4x32-10 (Salmon et al.,
+ * SC 2011) at counter (j / 4, i / 4, b Hq + h, offset) with key = seed (low
+ * word first), kept iff the byte is below T; LSE is that of the undropped
+ * probabilities.  The backward must get the same seed and offset.  The
+ * arguments are those of fa_fwd / fa_bwd plus dropout_p in [0, 1), seed
+ * and offset; T = 256 (p < 1/512) runs the plain kernels, and p so close to
+ * 1 that T = 0 is FA_ERR_INVALID_ARG.  d is 64 or 128; dense batches only.
+ */
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int Nq, int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3],
+                   const int64_t k_stride[3], const int64_t v_stride[3],
+                   const int64_t o_stride[3], int dtype, float softmax_scale, int causal,
+                   int window_left, int window_right, float dropout_p, uint64_t seed,
+                   uint32_t offset, void* stream);
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                   const int64_t q_stride[3], const int64_t k_stride[3],
+                   const int64_t v_stride[3], const int64_t o_stride[3],
+                   const int64_t do_stride[3], const int64_t dq_stride[3],
+                   const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
+                   float softmax_scale, int causal, int window_left, int window_right,
+                   float dropout_p, uint64_t seed, uint32_t offset, void* stream);
+
+/*
  * Forward on FP8 inputs: q, k, v hold float8_e4m3fn values (one byte each;
  * "optimizing-attention-flash", Workflow 3: inputs cast to float8_e4m3fn and
  * passed to the same attention call), o is bf16, lse fp32 [B, Hq, Nq].

@@ -1,0 +1,74 @@
+"""GPU parity of the forward and backward with dropout against the fp64 oracle.
+
+The kernels and the oracle draw the keep bits independently from Philox4x32-10
+(pinned to its published known-answer vectors on the oracle side); a single
+differing bit moves O by a whole term, so the O and gradient bars below also
+check that every keep bit agrees.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_143_b200 as fa
+import oracle
+from seeded_inputs import make_qkv
+from tests.parity import check_grad, check_lse, check_o, to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+CASES = [
+    # B, Nq, Nk, Hq, Hkv, d, dtype, causal, window, p, seed, offset
+    (2, 300, 300, 4, 2, 64, torch.float16, False, (-1, -1), 0.1, 1234, 0),
+    (1, 257, 257, 4, 4, 128, torch.bfloat16, True, (-1, -1), 0.5, 0xDEADBEEF12345678, 7),
+    (1, 200, 333, 2, 1, 64, torch.bfloat16, False, (40, 20), 0.25, 99, 3),
+    (2, 129, 129, 2, 2, 128, torch.float16, True, (-1, -1), 0.3, 5, 1),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "d%d_p%g_c%d" % (c[5], c[9], c[7]))
+def test_dropout_fwd_bwd_match_oracle(case):
+    B, Nq, Nk, Hq, Hkv, d, dtype, causal, window, p, seed, offset = case
+    q, k, v, do = make_qkv(B, Nq, Nk, Hq, Hkv, d, dtype, 80, with_dout=True)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    scale = d ** -0.5
+    kw = dict(softmax_scale=scale, causal=causal, window_size=window, dropout_p=p, seed=seed,
+              offset=offset)
+    o, lse = fa.fa_fwd(qd, kd, vd, **kw)
+    dq, dk, dv = fa.fa_bwd(dod, qd, kd, vd, o, lse, **kw)
+    torch.cuda.synchronize()
+    assert fa.get_device_error() == fa.FA_OK
+    T = oracle.dropout_keep_threshold(p)
+    o_ref, lse_ref = oracle.attention_fwd_dropout(to64(q), to64(k), to64(v), scale, T, seed,
+                                                  offset, causal, window)
+    check_o(o, o_ref, dtype)
+    check_lse(lse, lse_ref)
+    # the backward from the kernel's own O (D = rowsum(dO o O) uses it)
+    gq, gk, gv, _, _ = oracle.attention_bwd_dropout(to64(q), to64(k), to64(v), to64(do), scale,
+                                                    T, seed, offset, causal, window)
+    check_grad(dq, gq, "dQ")
+    check_grad(dk, gk, "dK")
+    check_grad(dv, gv, "dV")
+
+
+def test_dropout_seed_and_offset_matter():
+    q, k, v = (t.to(DEV) for t in make_qkv(1, 128, 128, 2, 2, 64, torch.bfloat16, 81))
+    a, la = fa.fa_fwd(q, k, v, dropout_p=0.2, seed=1, offset=0)
+    b, lb = fa.fa_fwd(q, k, v, dropout_p=0.2, seed=1, offset=0)
+    c, _ = fa.fa_fwd(q, k, v, dropout_p=0.2, seed=2, offset=0)
+    e, _ = fa.fa_fwd(q, k, v, dropout_p=0.2, seed=1, offset=1)
+    plain, lp = fa.fa_fwd(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)                 # deterministic for one seed and offset
+    assert not torch.equal(a, c) and not torch.equal(a, e)
+    assert torch.equal(la, lp)               # LSE ignores dropout
+    z, _ = fa.fa_fwd(q, k, v, dropout_p=1e-4, seed=3)  # T = 256: nothing dropped
+    assert torch.equal(z, plain)
+
+
+def test_dropout_rejects_p_near_one():
+    q, k, v = (t.to(DEV) for t in make_qkv(1, 64, 64, 1, 1, 64, torch.bfloat16, 82))
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_fwd(q, k, v, dropout_p=0.999)
+    assert e.value.status == fa.FA_ERR_INVALID_ARG
