@@ -80,8 +80,8 @@ def load_peaks():
 
 # the sources each profiled kernel is compiled from (device code only)
 KERNEL_SOURCES = {
-    "fa_bwd_main_kernel": ("fa_bwd.cuh", "fa_exp2.cuh", "fa_ptx.cuh"),
-    "fa_fwd_kernel": ("fa_fwd.cuh", "fa_exp2.cuh", "fa_ptx.cuh"),
+    "fa_bwd_main_kernel": ("fa_bwd.cuh", "fa_dropout.cuh", "fa_exp2.cuh", "fa_ptx.cuh"),
+    "fa_fwd_kernel": ("fa_fwd.cuh", "fa_dropout.cuh", "fa_exp2.cuh", "fa_ptx.cuh"),
 }
 
 
@@ -440,6 +440,18 @@ def run_ours(args):
                               "frac_of_fp8_peak": round(tf8 / (2 * peak), 4),
                               "frac_of_bf16_peak": round(tf8 / peak, 4)}
             del fq, fk, fv, fo, fl
+        # the main workload with dropout p = 0.1 (keep bits from the in-kernel
+        # generator): forward and backward, counted FLOPs as without dropout
+        dkw = dict(kw, dropout_p=0.1, seed=1234, offset=0)
+        dfms = time_steps(lambda _: fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **dkw), 10, 3, flush,
+                          stream)
+        dbms = time_steps(lambda _: fa.fa_bwd(dod, qd, kd, vd, o, lse, dq=dq, dk=dk, dv=dv,
+                                              workspace=ws, **dkw), 10, 3, flush, stream)
+        dfm, dbm = statistics.median(dfms), statistics.median(dbms)
+        table[w.name + "_dropout0.1"] = {"fwd_ms_median": round(dfm, 4),
+                                         "fwd_tflops": round(f_fwd / (dfm / 1e3) / 1e12, 1),
+                                         "bwd_ms_median": round(dbm, 4),
+                                         "bwd_tflops": round(2.5 * f_fwd / (dbm / 1e3) / 1e12, 1)}
         # the main workload's forward and backward separately
         fms = time_steps(lambda _: fa.fa_fwd(qd, kd, vd, out=o, lse=lse, **kw), 10, 3, flush,
                          stream)
