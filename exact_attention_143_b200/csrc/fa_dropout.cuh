@@ -34,13 +34,13 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
       k0 += 0x9E3779B9u;
       k1 += 0xBB67AE85u;
     }
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-    const uint32_t y0 = hi1 ^ c1 ^ k0, y2 = hi0 ^ c3 ^ k1;
+    const uint64_t p0 = uint64_t(0xD2511F53u) * c0;  // one 32 x 32 -> 64-bit product each
+    const uint64_t p1 = uint64_t(0xCD9E8D57u) * c2;
+    const uint32_t y0 = uint32_t(p1 >> 32) ^ c1 ^ k0, y2 = uint32_t(p0 >> 32) ^ c3 ^ k1;
     c0 = y0;
-    c1 = lo1;
+    c1 = uint32_t(p1);
     c2 = y2;
-    c3 = lo0;
+    c3 = uint32_t(p0);
   }
   return make_uint4(c0, c1, c2, c3);
 }
@@ -49,34 +49,36 @@ __device__ __forceinline__ uint32_t word_of(const uint4& w, int k) {
   return k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
 }
 
-// Forward: the keep bytes of query row i for the 16 key groups (64 keys) that
-// start at key jg0 (a multiple of 4): word (i mod 4) of each group's output,
-// out[g] for keys jg0 + 4g .. + 3 (byte k = key jg0 + 4g + k).  The four
-// lanes of a 4-row group (lanes 4t .. 4t + 3 hold rows i with the same i / 4)
-// share the generator calls: each computes four of the sixteen and the words
-// go to their rows in four shuffle rounds.
-__device__ __forceinline__ void dropout_row_words(const DropoutParams& dp, uint32_t bh, int i,
-                                                  int jg0, uint32_t (&out)[16]) {
+// Forward, four key groups at a time: word (i mod 4) of the generator output
+// of groups jg0/4 + 4k .. + 3 (keys jg0 + 16k .. + 15), out[m] for group 4k + m.
+// The four lanes of a 4-row group each make one of the four calls and pass
+// the words to their rows in four shuffle rounds.
+__device__ __forceinline__ void dropout_row_words4(const DropoutParams& dp, uint32_t bh, int i,
+                                                   int jg0, int k, uint32_t (&out)[4]) {
   const int lane = threadIdx.x & 31, q = lane & 3;
   const int base = lane & ~3;
+  const uint4 w = philox4x32_10(uint32_t((jg0 >> 2) + 4 * k + q), uint32_t(i >> 2), bh, dp.offset,
+                                dp.seed_lo, dp.seed_hi);
+  uint32_t got[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    // this lane's call: group 4k + q
-    const uint4 w = philox4x32_10(uint32_t((jg0 >> 2) + 4 * k + q), uint32_t(i >> 2), bh,
-                                  dp.offset, dp.seed_lo, dp.seed_hi);
-    uint32_t got[4];
+  for (int t = 0; t < 4; ++t)
+    got[t] = __shfl_sync(0xffffffffu, word_of(w, (q + t) & 3), base | ((q - t) & 3));
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      // send word (q + t) mod 4 of group 4k + q; receive word q of group
-      // 4k + ((q - t) mod 4) from the lane that owns it
-      got[t] = __shfl_sync(0xffffffffu, word_of(w, (q + t) & 3), base | ((q - t) & 3));
-    }
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int t = (q - m) & 3;  // round in which group 4k + m arrived
-      out[4 * k + m] = t == 0 ? got[0] : (t == 1 ? got[1] : (t == 2 ? got[2] : got[3]));
-    }
+  for (int m = 0; m < 4; ++m) {
+    const int t = (q - m) & 3;
+    out[m] = t == 0 ? got[0] : (t == 1 ? got[1] : (t == 2 ? got[2] : got[3]));
   }
+}
+
+// 0xFF in each byte of `word` that is below T (T in 1..255), 0x00 elsewhere.
+__device__ __forceinline__ uint32_t keep_bytes(uint32_t word, uint32_t T) {
+  return __vcmpltu4(word, T * 0x01010101u);
+}
+
+// A mask for a packed pair of 16-bit values: the low half from byte b of
+// `m`, the high half from byte b + 1 (b = 0 or 2).
+__device__ __forceinline__ uint32_t pair_mask(uint32_t m, int b) {
+  return __byte_perm(m, 0u, b == 0 ? 0x1100u : 0x3322u);
 }
 
 // Backward: the keep bytes of key row j for 16 query groups (64 queries)

@@ -477,11 +477,17 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
-        uint32_t kw[16];  // dropout keep bytes of this row for the half's 64 keys
-        if constexpr (DROP)
-          dropout_row_words(p.drop, uint32_t(b * p.Hq + h), row, key0 + 64 * half, kw);
+        uint32_t kw4[4];  // dropout keep bytes of the current 16 keys
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
+          // with dropout, the keep bytes of keys 64 half + 16 (c / 8) .. + 15
+          // (this row's word of four generator outputs) are drawn just before
+          // the eight pairs that use them
+          if constexpr (DROP) {
+            if ((c & 7) == 0)
+              dropout_row_words4(p.drop, uint32_t(b * p.Hq + h), row, key0 + 64 * half, c >> 3,
+                                 kw4);
+          }
           const int cc = 32 * half + c;  // column pair
           const float2 x = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), sc2, nb2);
           float2 pv;
@@ -491,12 +497,12 @@ __global__ void __launch_bounds__(352, 1)
             pv.x = fast_exp2(x.x);
             pv.y = fast_exp2(x.y);
           }
-          lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);
-          if constexpr (DROP) {  // l keeps the undropped sum
-            pv.x *= keep_of(kw[c >> 1], (c & 1) * 2, p.drop.T);
-            pv.y *= keep_of(kw[c >> 1], (c & 1) * 2 + 1, p.drop.T);
-          }
+          lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);  // l keeps the undropped sum
           pk[c] = pack2<BF16>(pv.x, pv.y);
+          if constexpr (DROP) {  // keys 2c, 2c + 1: bytes 2 (c & 1), + 1 of group c / 2
+            const uint32_t kb = keep_bytes(kw4[(c >> 1) & 3], p.drop.T);
+            pk[c] &= pair_mask(kb, (c & 1) * 2);
+          }
         }
         // P_t V_{j-1}, the last reader of P_t, must be complete before P_t is
         // rewritten.  It is awaited on its own barrier: the completion of
