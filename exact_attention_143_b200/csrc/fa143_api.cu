@@ -702,15 +702,19 @@ int sm_count() {
 }
 
 // Splits of the key tiles of every (sequence, kv head): enough CTAs for about
-// two per SM when the batch alone does not provide them, at least one tile each.
+// four per SM (two run at a time) when the batch alone does not provide them,
+// and no split longer than 32 tiles, so that long sequences do not leave a
+// tail of lone CTAs; at least one tile each.
 int decode_splits(int B, int Hkv, int max_tiles, int requested, int& tiles_per_split) {
   int splits;
   if (requested > 0) {
     splits = requested;
   } else {
     const int64_t units = int64_t(B) * Hkv;
-    const int64_t want = 2 * int64_t(sm_count());
-    splits = units >= want ? 1 : int((want + units - 1) / units);
+    const int64_t want = 4 * int64_t(sm_count());
+    const int by_fill = units >= want ? 1 : int((want + units - 1) / units);
+    const int by_length = (max_tiles + 31) / 32;
+    splits = std::max(by_fill, by_length);
   }
   splits = std::max(1, std::min(splits, max_tiles));
   tiles_per_split = (max_tiles + splits - 1) / splits;
@@ -736,7 +740,7 @@ int check_paged_shape(int B, int Nq, int Hq, int Hkv, int d, int page_size, int 
 }
 
 // 4-D map over a paged cache [num_pages, P, Hkv, d] (innermost first: d, Hkv,
-// P, pages), box of 64 columns x 1 head x min(P, 128) rows x 1 page.
+// P, pages), box of 64 columns x 1 head x min(P, 64) rows x 1 page.
 int make_cache_map(CUtensorMap* map, const void* ptr, const int64_t st[3], int num_pages, int P,
                    int Hkv, int d, int dtype) {
   EncodeTiledFn enc = get_encode_fn();
@@ -746,7 +750,7 @@ int make_cache_map(CUtensorMap* map, const void* ptr, const int64_t st[3], int n
   const int64_t sh = Hkv > 1 ? st[2] : 8;
   cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(Hkv), cuuint64_t(P), cuuint64_t(num_pages)};
   cuuint64_t strides[3] = {cuuint64_t(sh) * 2, cuuint64_t(stok) * 2, cuuint64_t(sp) * 2};
-  cuuint32_t box[4] = {64, 1, cuuint32_t(std::min(P, 128)), 1};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(std::min(P, 64)), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map,
                    dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -791,14 +795,15 @@ int launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMa
   using Cfg = fa::DecCfg<D>;
   auto kern = fa::fa_decode_kernel<D, BF16>;
   static bool attr_done = false;  // per instantiation and process
-  if (!attr_done) {
+  if (!attr_done) {  // room for the largest query tile (128 rows)
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
+                             Cfg::smem_bytes(128)) != cudaSuccess)
       return FA_ERR_CUDA;
     attr_done = true;
   }
+  const int smem = Cfg::smem_bytes((prm.R + 7) & ~7);
   dim3 grid(unsigned(prm.n_splits), unsigned(prm.Hkv), unsigned(prm.B));
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
+  kern<<<grid, Cfg::kThreads, smem, st>>>(mq, mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (prm.n_splits > 1) {
     const int64_t rows = int64_t(prm.B) * prm.Hq * prm.Nq;
@@ -818,7 +823,8 @@ size_t fa_fwd_paged_workspace_size(int B, int Nq, int Hq, int Hkv, int d, int pa
                         -1))
     return 0;
   const int max_tiles =
-      int((int64_t(max_pages_per_seq) * page_size + 127) / 128);
+      int((int64_t(max_pages_per_seq) * page_size + fa::DecCfg<128>::kKeys - 1) /
+          fa::DecCfg<128>::kKeys);
   int tps = 0;
   const int splits = decode_splits(B, Hkv, max_tiles, num_splits, tps);
   return paged_workspace_bytes(B, Hkv, (Hq / Hkv) * Nq, d, splits);
@@ -858,7 +864,8 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
       overlaps_span(tv, lse, lse_bytes) || overlaps_span(to, lse, lse_bytes))
     return FA_ERR_INVALID_ARG;
 
-  const int max_tiles = int((int64_t(max_pages_per_seq) * page_size + 127) / 128);
+  const int max_tiles = int((int64_t(max_pages_per_seq) * page_size + fa::DecCfg<128>::kKeys - 1) /
+                            fa::DecCfg<128>::kKeys);
   int tps = 0;
   const int splits = decode_splits(B, Hkv, max_tiles, num_splits, tps);
   const size_t need = paged_workspace_bytes(B, Hkv, G * Nq, d, splits);

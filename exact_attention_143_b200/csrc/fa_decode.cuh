@@ -15,26 +15,29 @@
 // byte, so the kernel is bound by HBM; its design goal is to keep enough page
 // loads in flight on every SM.
 //
-// B200 mapping:
+// B200 mapping (two CTAs per SM, so two independent load pipelines):
 //   grid (split, kv head g, sequence b).  The visible key tiles of a sequence
-//   are cut into splits of `tiles_per_split` 128-key tiles, so short batches
+//   are cut into splits of `tiles_per_split` 64-key tiles, so short batches
 //   still fill the 148 SMs; a combine kernel merges the splits.
 //   rows: the G query heads of kv head g times the Nq queries (r = h' Nq + i)
-//   form one 128-row tile (rows past G Nq are zero), loaded by one TMA box.
-//   warp 4   TMA: the query tile once, then a ring of K and V tiles, each
-//            assembled from 128 / min(P, 128) page boxes issued by as many
-//            lanes; a page past the sequence is fetched at an out-of-range
-//            page coordinate, which TMA fills with zeros.
-//   warp 5   tcgen05 issuer: S = Q K^T into one of two tensor-memory
-//            regions, O += P V with P read from one of two regions of its own.
+//   form the query tile, loaded by one TMA box per 64-column chunk; a chunk
+//   holds R rounded up to 8 rows (the rest zero), which keeps shared memory
+//   small enough for two CTAs per SM.
+//   warp 4   TMA: the query tile once, then a ring of K and V tiles of 64
+//            keys, each assembled from 64 / min(P, 64) page boxes issued by as
+//            many lanes; a page past the sequence is fetched at an
+//            out-of-range page coordinate, which TMA fills with zeros.
+//   warp 5   tcgen05 issuer: S = Q K^T (N = 64) into one of two 64-column
+//            regions, O += P V with P over S.
 //   warps 0-3 softmax: thread r owns row r (tensor-memory lane r); masks,
 //            running max / sum with the lazy O rescale.  P(j) is written once
 //            P V(j-2), the last reader of its region, is done, and O is
 //            rescaled once P V(j-1) is done, each awaited on the barrier
 //            committed with that MMA.
-//            Thread r also clears V row r of the tile when its key lies past
-//            the cache length: a partly filled page holds whatever the caller
-//            left there, and 0 * NaN would poison O.
+//            Thread r < 64 also clears V row r of the tile when its key lies
+//            past the cache length: a partly filled page holds whatever the
+//            caller left there, and 0 * NaN would poison O.
+// Tensor memory (256 columns): S regions at 0 and 64, O at 128.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -68,17 +71,20 @@ struct DecodeParams {
 
 template <int D>
 struct DecCfg {
-  static constexpr int kChunk = 128 * 64 * 2;     // one 128-row x 64-column swizzled chunk
-  static constexpr int kTileBytes = 128 * D * 2;  // a 128-row tile
-  static constexpr int kStages = D == 64 ? 6 : 3;  // K+V ring depth
+  static constexpr int kKeys = 64;                  // keys per K/V tile
+  static constexpr int kKVChunk = kKeys * 128;      // 64 rows x 64 columns, 128-byte swizzled
+  static constexpr int kTileBytes = kKeys * D * 2;  // one K or one V tile
+  static constexpr int kStages = D == 64 ? 6 : 3;   // K+V ring depth
   static constexpr int kThreads = 192;
-  static constexpr int kSmemQ = 1024;  // barriers and the tensor-memory slot below
-  static constexpr int kSmemK = kSmemQ + kTileBytes;
-  static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kSmemV + kStages * kTileBytes + 1024;  // + alignment slack
-  static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColO = 256;
-  static constexpr uint32_t kColP = 256 + D;  // P(j) at kColP + 64 (j % 2)
+  static constexpr int kSmemQ = 1024;               // barriers and the tensor-memory slot below
+  static constexpr uint32_t kTmemCols = 256;        // two CTAs share an SM's 512 columns
+  static constexpr uint32_t kColO = 128;            // S regions at 0 and 64, O at 128
+  // shared memory of a launch whose query tile has r_pad rows per column chunk:
+  // Q, then the K ring and the V ring (each 1024-byte aligned), + alignment slack
+  __host__ __device__ static constexpr int q_bytes(int r_pad) { return (D / 64) * r_pad * 128; }
+  __host__ __device__ static constexpr int k_off(int r_pad) { return (kSmemQ + q_bytes(r_pad) + 1023) / 1024 * 1024; }
+  __host__ __device__ static constexpr int v_off(int r_pad) { return k_off(r_pad) + kStages * kTileBytes; }
+  __host__ __device__ static constexpr int smem_bytes(int r_pad) { return v_off(r_pad) + kStages * kTileBytes + 1024; }
 };
 
 // Visible key range [lo, hi] of query i of a sequence holding Nk keys.
@@ -91,15 +97,22 @@ __device__ __forceinline__ void decode_key_range(int i, int Nq, int Nk, int caus
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using Cfg = DecCfg<D>;
   constexpr int S = Cfg::kStages;
+  constexpr int KT = Cfg::kKeys;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
+  // the query tile holds r_pad rows per 64-column chunk (R rounded up to 8);
+  // the MMA reads 128 rows from each chunk base, the rows past r_pad landing
+  // in this CTA's K/V ring: they only feed output rows that are never stored
+  const int r_pad = (p.R + 7) & ~7;
+  const int q_chunk = r_pad * 128;
+  const int off_k = Cfg::k_off(r_pad), off_v = Cfg::v_off(r_pad);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
   const uint32_t bar_q = smem_u32(&bars[0]);
@@ -119,15 +132,15 @@ __global__ void __launch_bounds__(192, 1)
   const int Nq = p.Nq;
   const int Nk = min(max(p.cache_seqlens[b], 0), p.max_pages * p.P);
 
-  // key tiles any row can see ([lo, hi] grows with the query index), and this
-  // split's share of them
+  // 64-key tiles any row can see ([lo, hi] grows with the query index), and
+  // this split's share of them
   int lo0, hi0, lo1, hi1;
   decode_key_range(0, Nq, Nk, p.causal, p.wl, p.wr, lo0, hi0);
   decode_key_range(Nq - 1, Nq, Nk, p.causal, p.wl, p.wr, lo1, hi1);
   int JLO = 0, JHI = 0;
   if (lo0 <= hi1 && Nk > 0) {
-    JLO = lo0 / 128;
-    JHI = hi1 / 128 + 1;
+    JLO = lo0 / KT;
+    JHI = hi1 / KT + 1;
   }
   const int j0 = JLO + split * p.tiles_per_split;
   const int j1 = min(JHI, j0 + p.tiles_per_split);
@@ -148,11 +161,11 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // query rows past R are zero (the MMA reads all 128 rows of the tile)
-  for (int idx = threadIdx.x; idx < (128 - p.R) * (D / 8); idx += blockDim.x) {
+  // query rows R .. r_pad - 1 of each chunk are zero
+  for (int idx = threadIdx.x; idx < (r_pad - p.R) * (D / 8); idx += blockDim.x) {
     const int row = p.R + idx / (D / 8), u = idx % (D / 8);  // 16-byte unit of the row
-    *reinterpret_cast<uint4*>(smem + Cfg::kSmemQ + (u / 8) * Cfg::kChunk + row * 128 +
-                              (u % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(smem + Cfg::kSmemQ + (u / 8) * q_chunk + row * 128 + (u % 8) * 16) =
+        make_uint4(0u, 0u, 0u, 0u);
   }
   fence_proxy_async_smem();
   __syncwarp();
@@ -169,7 +182,7 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ TMA producer
     // The whole warp runs the loop.  Lane bx reads the page id of box bx of
     // the tile before the wait for the free stage and then issues that box's
-    // copies, so the copies of one tile leave from up to 16 threads.
+    // copies, so the copies of one tile leave from up to 8 threads.
     if (n > 0) {
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -177,16 +190,16 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmV);
         mbar_arrive_expect_tx(bar_q, uint32_t(p.R * 128 * (D / 64)));
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sbase + Cfg::kSmemQ + c * Cfg::kChunk, &tmQ, bar_q, c * 64, 0, g * p.G, b);
+          tma_load_4d(sbase + Cfg::kSmemQ + c * q_chunk, &tmQ, bar_q, c * 64, 0, g * p.G, b);
       }
-      const int rows_per_box = min(p.P, 128);
-      const int boxes = 128 / rows_per_box;  // at most 16 (pages of 8 or more rows)
+      const int rows_per_box = min(p.P, KT);
+      const int boxes = KT / rows_per_box;  // at most 8 (pages of 8 or more rows)
       const int* bt = p.block_table + int64_t(b) * p.bt_stride;
       const int n_seq_pages = (Nk + p.P - 1) / p.P;
       bool ok = true;
       for (int jj = 0; jj < n && ok; ++jj) {
         const int s = jj % S, u = jj / S;
-        const int key0 = (j0 + jj) * 128;
+        const int key0 = (j0 + jj) * KT;
         // a page the sequence does not hold is read at an out-of-range page
         // coordinate: TMA delivers zeros for it
         int my_page = p.num_pages;
@@ -198,16 +211,14 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
         if (lane == 0) mbar_arrive_expect_tx(bar_full(s), 2 * Cfg::kTileBytes);
         __syncwarp();
-        // lane bx copies the boxes of its own page: a single issuing thread
-        // cannot keep the copy engine busy with boxes this small
         if (lane < boxes) {
           const int tok = (key0 + lane * rows_per_box) % p.P;
           const uint32_t row_off = uint32_t(lane * rows_per_box * 128);
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_4d(sbase + Cfg::kSmemK + s * Cfg::kTileBytes + c * Cfg::kChunk + row_off,
-                        &tmK, bar_full(s), c * 64, g, tok, my_page);
-            tma_load_4d(sbase + Cfg::kSmemV + s * Cfg::kTileBytes + c * Cfg::kChunk + row_off,
-                        &tmV, bar_full(s), c * 64, g, tok, my_page);
+            tma_load_4d(sbase + off_k + s * Cfg::kTileBytes + c * Cfg::kKVChunk + row_off, &tmK,
+                        bar_full(s), c * 64, g, tok, my_page);
+            tma_load_4d(sbase + off_v + s * Cfg::kTileBytes + c * Cfg::kKVChunk + row_off, &tmV,
+                        bar_full(s), c * 64, g, tok, my_page);
           }
         }
         __syncwarp();
@@ -215,27 +226,28 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    // S_j goes to region j % 2 and P_j to P region j % 2; S_{j+2} is issued
-    // after P_j V_j, so two S tiles run ahead of the softmax.
+    // S_j goes to region j % 2 and P_j over it; S_{j+2} is issued after
+    // P_j V_j, so two S tiles run ahead of the softmax.
     if (n > 0) {
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
       };
-      constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);            // K-major tiles
-      constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kChunk, 1024);  // V, MN-major
-      const uint32_t idesc_qk = make_idesc_f16(BF16, 128, 128, false, false) | (p.qk_negate << 13);
+      constexpr uint64_t kDescK = sdesc_sw128_const(16, 1024);              // K-major tiles
+      constexpr uint64_t kDescMN = sdesc_sw128_const(Cfg::kKVChunk, 1024);  // V, MN-major
+      const uint32_t idesc_qk = make_idesc_f16(BF16, 128, KT, false, false) | (p.qk_negate << 13);
       const uint32_t idesc_pv = make_idesc_f16(BF16, 128, D, false, true);
       const uint64_t dQ = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
-      const uint64_t dK0 = sdesc_at(kDescK, sbase + Cfg::kSmemK);
-      const uint64_t dV0 = sdesc_at(kDescMN, sbase + Cfg::kSmemV);
+      const uint64_t dK0 = sdesc_at(kDescK, sbase + off_k);
+      const uint64_t dV0 = sdesc_at(kDescMN, sbase + off_v);
       auto issue_s = [&](int jj) {
         const int s = jj % S;
         const uint64_t kb = dK0 + uint64_t((s * Cfg::kTileBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = uint64_t(((kk >> 2) * Cfg::kChunk + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + (jj & 1) * 128, dQ + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
+            const uint64_t qo = uint64_t(((kk >> 2) * q_chunk + (kk & 3) * 32) >> 4);
+            const uint64_t ko = uint64_t(((kk >> 2) * Cfg::kKVChunk + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + (jj & 1) * 64, dQ + qo, kb + ko, idesc_qk, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_sfull(jj & 1));
         }
@@ -254,8 +266,8 @@ __global__ void __launch_bounds__(192, 1)
         const uint64_t vb = dV0 + uint64_t((s * Cfg::kTileBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts(tmem + Cfg::kColO, tmem + Cfg::kColP + (jj & 1) * 64 + kk * 8,
+          for (int kk = 0; kk < KT / 16; ++kk)  // P: 16 keys of 16-bit values = 8 columns
+            mma_ts(tmem + Cfg::kColO, tmem + (jj & 1) * 64 + kk * 8,
                    vb + uint64_t((kk * 16 * 128) >> 4), idesc_pv, (kk > 0 || jj > 0) ? 1u : 0u);
           mma_commit(bar_odone(jj & 1));
           mma_commit(bar_empty(s));
@@ -285,18 +297,18 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       const int s = jj % S;
-      const int key0 = (j0 + jj) * 128;
-      const uint32_t tS = tmem + lane_base + (jj & 1) * 128;
+      const int key0 = (j0 + jj) * KT;
+      const uint32_t tS = tmem + lane_base + (jj & 1) * 64;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(jj & 1), (jj >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
       // V row r of this tile holds key key0 + r: clear it when that key is past
       // the cache length (the S MMA has completed, so the tile has landed)
-      if (key0 + r >= Nk) {
+      if (r < KT && key0 + r >= Nk) {
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          uint4* vrow = reinterpret_cast<uint4*>(smem + Cfg::kSmemV + s * Cfg::kTileBytes +
-                                                 c * Cfg::kChunk + r * 128);
+          uint4* vrow = reinterpret_cast<uint4*>(smem + off_v + s * Cfg::kTileBytes +
+                                                 c * Cfg::kKVChunk + r * 128);
 #pragma unroll
           for (int u = 0; u < 8; ++u) vrow[u] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -305,31 +317,27 @@ __global__ void __launch_bounds__(192, 1)
       float alpha = 1.f;
       bool grow = false;
       if (warp_has_rows) {
-        uint32_t sr0[32], sr1[32], sr2[32], sr3[32];
+        uint32_t sr0[32], sr1[32];
         tmem_ld32(tS + 0, sr0);
         tmem_ld32(tS + 32, sr1);
-        tmem_ld32(tS + 64, sr2);
-        tmem_ld32(tS + 96, sr3);
         tmem_wait_ld();
-        float sv[128];
+        float sv[64];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           sv[c] = __uint_as_float(sr0[c]);
           sv[32 + c] = __uint_as_float(sr1[c]);
-          sv[64 + c] = __uint_as_float(sr2[c]);
-          sv[96 + c] = __uint_as_float(sr3[c]);
         }
-        const bool need_mask = (lo_i > key0) || (hi_i < key0 + 127);
+        const bool need_mask = (lo_i > key0) || (hi_i < key0 + KT - 1);
         if (__any_sync(0xffffffffu, need_mask)) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < 64; ++c)
             sv[c] = (key0 + c >= lo_i && key0 + c <= hi_i) ? sv[c] : -INFINITY;
         }
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
 #pragma unroll
-        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sc;
@@ -345,26 +353,22 @@ __global__ void __launch_bounds__(192, 1)
         const float2 nb2 = make_float2(-base, -base);
         float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
-        // P(j) replaces P(j-2) once P V(j-2) is done
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {  // key pair
+          const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nb2);
+          const float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          lsum[c & 3] = __fadd2_rn(lsum[c & 3], pv);
+          pk[c] = pack2<BF16>(pv.x, pv.y);
+        }
+        // P(j) goes over S(j) (already read) once P V(j-2), the last reader of
+        // this region's P, is done
         if (jj >= 2) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(jj & 1), ((jj >> 1) + 1) & 1, wc));
           if (!ok) break;
           tc_fence_after();
         }
-        const uint32_t tP = tmem + lane_base + Cfg::kColP + (jj & 1) * 64;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int cc = 32 * half + c;  // column pair
-            const float2 x = __ffma2_rn(make_float2(sv[2 * cc], sv[2 * cc + 1]), sc2, nb2);
-            const float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-            lsum[cc & 3] = __fadd2_rn(lsum[cc & 3], pv);
-            pk[c] = pack2<BF16>(pv.x, pv.y);
-          }
-          tmem_st32(tP + 32 * half, pk);
-        }
+        tmem_st32(tS, pk);
         const float2 ls2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
         l += ls2.x + ls2.y;
       }
@@ -389,7 +393,6 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(bar_pfull(jj & 1));
     }
-    // epilogue: this split's O / l and its log2-sum-exp2, or the final O, LSE
     // every P V done: the last two, one per region (earlier ones were awaited)
     for (int jl = max(0, n - 2); jl < n && ok; ++jl)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(jl & 1), (jl >> 1) & 1, wc));
