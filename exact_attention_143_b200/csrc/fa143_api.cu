@@ -168,6 +168,11 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::kSmemBytes) != cudaSuccess)
       return FA_ERR_CUDA;
+    // the kernel moves registers between warpgroups (setmaxnreg); that is only
+    // sound when it is launched with exactly the planned count per thread
+    cudaFuncAttributes fattr{};
+    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess || fattr.numRegs != Cfg::kRegsLaunch)
+      return FA_ERR_CUDA;
     attr_done = true;
   }
   dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));

@@ -22,6 +22,8 @@
 //                tensor memory when m grows by more than 2^8 (exact: the
 //                final O / l uses the same m), and runs the epilogue
 //                (O / l to HBM, LSE = ln 2 * (m + log2 l)).
+//   warp 11      idle; it completes warpgroup 2, whose registers move to the
+//                softmax warpgroups (setmaxnreg) after the prologue.
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 at 256
 // and 256 + d.  With d = 64 the 128 spare columns hold P_0 and P_1, so
 // S_t(j+1) is computed while the softmax of S_t(j) is still running; with
@@ -65,7 +67,13 @@ struct FwdCfg {
   static constexpr int kChunk = 128 * 64 * 2;       // one 128-row x 64-column swizzled chunk
   static constexpr int kTileBytes = 128 * D * 2;    // a 128-row tile
   static constexpr int kStages = D == 64 ? 4 : 2;   // K ring and V ring depth
-  static constexpr int kThreads = 352;
+  static constexpr int kThreads = 384;               // 3 warpgroups, warp 11 idle
+  // registers per thread: at launch, and after the split that moves them from
+  // the control warpgroup (MMA issue, TMA) to the two softmax warpgroups;
+  // 128 * (2 * kRegsSoftmax + kRegsCtl) must equal kThreads * kRegsLaunch
+  static constexpr int kRegsLaunch = 168;
+  static constexpr int kRegsSoftmax = 216;
+  static constexpr int kRegsCtl = 72;
   static constexpr int kSmemQ = 1024;
   static constexpr int kSmemK = kSmemQ + kTiles * kTileBytes;
   static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
@@ -100,7 +108,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 template <int D, bool BF16, bool DROP = false>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Cfg = FwdCfg<D>;
@@ -200,7 +208,13 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 10) {
+  static_assert(128 * (2 * Cfg::kRegsSoftmax + Cfg::kRegsCtl) == Cfg::kThreads * Cfg::kRegsLaunch,
+                "register split must add up to the launch budget");
+  if (warp >= 8) {
+   // warpgroup 2 (warp 11 idle) hands registers to the softmax warpgroups;
+   // the instruction is executed by all four warps before they diverge
+   regs_dec<Cfg::kRegsCtl>();
+   if (warp == 10) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && JHI > JLO) {
       tma_prefetch_desc(&tmQ);
@@ -399,8 +413,10 @@ __global__ void __launch_bounds__(352, 1)
         }
       }
     }
+   }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    regs_inc<Cfg::kRegsSoftmax>();
     const int t = warp >> 2;          // query tile of this warpgroup
     const int r = threadIdx.x & 127;  // row within the tile == tensor-memory lane
     const int row = mblock * 256 + t * 128 + r;
