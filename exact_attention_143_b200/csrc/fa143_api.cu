@@ -13,6 +13,7 @@
 
 #include "fa143.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_aux.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd256.cuh"
