@@ -393,11 +393,15 @@ def run_ours(args):
             to = torch.empty_like(tq)
             tl = torch.empty(tw.batch, tw.q_heads, tw.seqlen_q, dtype=torch.float32, device=dev)
             tkw = dict(softmax_scale=tw.softmax_scale, causal=tw.causal, window_size=tw.window)
-            tms = time_steps(lambda _: fa.fa_fwd(tq, tk, tv, out=to, lse=tl, **tkw), 20, 3, flush,
-                             stream)
+            # 10 warm-ups, then 50 timed launches with L2 flushed before each
+            # (the headline figures), and 50 more back to back with L2 warm
+            fwd1 = lambda _: fa.fa_fwd(tq, tk, tv, out=to, lse=tl, **tkw)  # noqa: E731
+            tms = time_steps(fwd1, 50, 10, flush, stream)
+            wms = time_steps(fwd1, 50, 0, lambda: None, stream)
             med = statistics.median(tms)
             tf = fwd_flops(tw) / (med / 1e3) / 1e12
             table[name] = {"fwd_ms_median": round(med, 4), "fwd_ms_min": round(min(tms), 4),
+                           "fwd_ms_median_warm_l2": round(statistics.median(wms), 4),
                            "fwd_tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
             del tq, tk, tv, to, tl
         # packed variable-length batch (no padding): forward and backward
