@@ -21,6 +21,8 @@
 
 namespace {
 
+int sm_count();  // streaming multiprocessors of the current device (cached)
+
 __device__ unsigned int g_device_error = 0u;
 
 uint64_t g_wait_limit_ns = 2000000000ull;
@@ -314,7 +316,12 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   prm.Nk = Nk;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
-  prm.n_mblocks = d == 256 ? (Nq + 127) / 128 : (Nq + 255) / 256;
+  // 256 query rows per CTA; a causal problem that would not fill the SMs runs
+  // one 128-row tile per CTA, which halves the longest CTA (the last query
+  // block sees the most keys).  The d = 256 kernel always takes 128 rows.
+  prm.mrows = 256;
+  if (d == 256 || (causal && int64_t(B) * Hq * ((Nq + 255) / 256) < sm_count())) prm.mrows = 128;
+  prm.n_mblocks = (Nq + prm.mrows - 1) / prm.mrows;
   prm.scale_log2 = scale_log2_of(softmax_scale);
   prm.qk_negate = softmax_scale < 0.f ? 1u : 0u;
   prm.causal = causal ? 1 : 0;

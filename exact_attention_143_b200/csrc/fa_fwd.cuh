@@ -7,7 +7,8 @@
 // attention is computed per block and the output is updated incrementally
 // with correct normalisation; matmul -> softmax -> matmul fused in one kernel).
 //
-// B200 mapping (one CTA = 256 query rows of one (batch, head)):
+// B200 mapping (one CTA = 256 query rows of one (batch, head); 128 rows, tile 1
+// idle, for causal problems too small to fill the SMs):
 //   warp 10      TMA producer: Q tiles once, then a ring of K and V tiles
 //                (128 keys x d each, 128-byte swizzle) with mbarrier hand-off.
 //   warps 8, 9   tcgen05 issuers: warp 8 issues S_t = Q_t K_j^T into tensor
@@ -45,7 +46,7 @@ struct FwdParams {
   float* lse;
   int64_t o_sb, o_ss, o_sh;  // element strides of O: batch, seq, head
   int B, Nq, Nk, Hq, Hkv;
-  int n_mblocks;             // ceil(Nq / 256)
+  int n_mblocks;             // ceil(Nq / mrows)
   float scale_log2;          // |softmax_scale| * log2(e)
   int causal, wl, wr;        // wl / wr: -1 = unbounded
   uint32_t qk_negate;        // 1 if softmax_scale < 0 (negate A in Q K^T)
@@ -59,6 +60,9 @@ struct FwdParams {
   const int* cu_k;
   int total_q, total_k;
   DropoutParams drop;  // used by the DROP instantiations only
+  // query rows per CTA: 256 (two tiles), or 128 (tile 1 idle) where fewer
+  // CTAs than SMs would otherwise run
+  int mrows;
 };
 
 template <int D>
@@ -154,14 +158,14 @@ __global__ void __launch_bounds__(384, 1)
     kstart = k0;
     bc = 0;
   }
-  if (mblock * 256 >= Nq) return;  // no query row of this sequence here (CTA-uniform)
+  if (mblock * p.mrows >= Nq) return;  // no query row of this sequence here (CTA-uniform)
 
   // K-tile range [jlo_t, jhi_t) of each query tile t (empty when jlo_t == jhi_t)
   auto tile_range = [&](int t, int& lo_j, int& hi_j) {
-    const int r0 = mblock * 256 + t * 128;
+    const int r0 = mblock * p.mrows + t * 128;
     lo_j = 0;
     hi_j = 0;
-    if (r0 < Nq) {
+    if (t * 128 < p.mrows && r0 < Nq) {
       const int r1 = min(r0 + 127, Nq - 1);
       int lo0, hi0, lo1, hi1;
       row_key_range(r0, Nq, Nk, p.causal, p.wl, p.wr, lo0, hi0);
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(sbase + Cfg::kSmemQ + t * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ, bar_q,
-                      c * 64, qstart + mblock * 256 + t * 128, h, bc);
+                      c * 64, qstart + mblock * p.mrows + t * 128, h, bc);
       bool ok = true;
       for (int j = JLO; j < JHI && ok; ++j) {
         const int idx = j - JLO, s = idx % S, u = idx / S;
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(384, 1)
     regs_inc<Cfg::kRegsSoftmax>();
     const int t = warp >> 2;          // query tile of this warpgroup
     const int r = threadIdx.x & 127;  // row within the tile == tensor-memory lane
-    const int row = mblock * 256 + t * 128 + r;
+    const int row = mblock * p.mrows + t * 128 + r;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tP = kSepP ? tmem + lane_base + Cfg::kColP + t * 64 : tS;
@@ -560,7 +564,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool has = (n > 0) && (l > 0.f);
       const float inv_l = has ? (DROP ? p.drop.scale : 1.f) / l : 0.f;
       const float lse = has ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const bool store = row < Nq;
+      const bool store = row < Nq && t * 128 < p.mrows;  // tile 1 idles at 128 rows
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + bc * p.o_sb + int64_t(qstart + row) * p.o_ss +
                        int64_t(h) * p.o_sh;
 #pragma unroll
