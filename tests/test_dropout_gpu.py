@@ -24,6 +24,9 @@ CASES = [
     (1, 257, 257, 4, 4, 128, torch.bfloat16, True, (-1, -1), 0.5, 0xDEADBEEF12345678, 7),
     (1, 200, 333, 2, 1, 64, torch.bfloat16, False, (40, 20), 0.25, 99, 3),
     (2, 129, 129, 2, 2, 128, torch.float16, True, (-1, -1), 0.3, 5, 1),
+    # enough heads to fill the SMs, so the causal forward keeps two query tiles
+    # per CTA (the smaller causal cases above take one)
+    (2, 300, 300, 40, 8, 64, torch.float16, True, (-1, -1), 0.2, 77, 2),
 ]
 
 

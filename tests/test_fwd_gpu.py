@@ -58,6 +58,15 @@ def test_lengths(Nq, Nk, causal):
     run_case(1, Nq, Nk, 2, 1, 64, torch.float16, causal, (-1, -1), seed=6)
 
 
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)], ids=["d64", "d128"])
+@pytest.mark.parametrize("window", [(-1, -1), (130, -1)], ids=["causal", "causal_w130"])
+def test_causal_full_grid_ragged(d, dtype, window):
+    # 2 x 40 heads x two 256-row blocks = 160 CTAs, enough to fill the SMs, so
+    # the kernel keeps two 128-row query tiles per CTA (smaller causal problems
+    # take one); the second block is ragged (rows 256-299)
+    run_case(2, 300, 300, 40, 8, d, dtype, True, window, seed=9)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (8, 1), (6, 2)])
 def test_gqa(Hq, Hkv):
     run_case(2, 260, 260, Hq, Hkv, 128, torch.bfloat16, True, (-1, -1), seed=7)
