@@ -36,7 +36,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
-            "fa_bwd_noalloc", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
+            "fa_bwd_noalloc", "fa_bwd_noalloc_scratch_bytes", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_fwd_paged_workspace_size", "fa_fwd_paged", "fa_fwd_fp8", "fa_fwd_dropout",
             "fa_bwd_dropout")
 
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_set_bwd_main_events.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [i64p] * 8 + [i, f, i, i, i, vp]
     lib.fa_bwd_noalloc.restype = i
+    lib.fa_bwd_noalloc_scratch_bytes.argtypes = []
+    lib.fa_bwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.fa_fwd_varlen.argtypes = [vp] * 7 + [i] * 8 + [i64p] * 4 + [i, f, i, i, i, vp]
     lib.fa_fwd_varlen.restype = i
     lib.fa_bwd_varlen.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [vp, vp] + [i] * 8 +
@@ -253,6 +255,7 @@ def fa_bwd_varlen(dout, q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_
     if workspace is None:
         workspace = torch.empty(bwd_workspace_size(B, int(max_seqlen_q), Hq, d), dtype=torch.uint8,
                                 device=dev)
+    _check_cuda(q, dq, dk, dv, workspace)
     wl, wr = window_size
     with torch.cuda.device(dev):
         rc = lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
@@ -21,11 +22,29 @@
 
 namespace {
 
-int sm_count();  // streaming multiprocessors of the current device (cached)
+int sm_count();  // streaming multiprocessors of the current device (cached per device)
 
 __device__ unsigned int g_device_error = 0u;
 
-uint64_t g_wait_limit_ns = 2000000000ull;
+// read by every launch, set by fa_set_wait_limit_ns from any host thread
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+// One-time set-up per device (per kernel instantiation): kernel attributes
+// such as the dynamic shared-memory opt-in apply to the current device only,
+// so a process that drives several devices needs them once on each.
+constexpr int kMaxDevices = 64;
+struct DeviceOnce {
+  std::atomic<uint8_t> done[kMaxDevices];  // static storage: starts at zero
+};
+template <typename F>
+int once_per_device(DeviceOnce& once, F&& setup) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (once.done[dev].load(std::memory_order_acquire)) return FA_OK;
+  const int rc = setup();  // idempotent: two threads may both run it
+  if (rc == FA_OK) once.done[dev].store(1, std::memory_order_release);
+  return rc;
+}
 cudaEvent_t g_bwd_ev_start = nullptr, g_bwd_ev_stop = nullptr;
 
 // ------------------------------------------------------------------ driver entry point
@@ -166,17 +185,20 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
                const fa::FwdParams& prm, cudaStream_t st) {
   using Cfg = fa::FwdCfg<D>;
   auto kern = fa::fa_fwd_kernel<D, BF16, DROP>;
-  static bool attr_done = false;  // per instantiation and process
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
-      return FA_ERR_CUDA;
-    // the kernel moves registers between warpgroups (setmaxnreg); that is only
-    // sound when it is launched with exactly the planned count per thread
-    cudaFuncAttributes fattr{};
-    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess || fattr.numRegs != Cfg::kRegsLaunch)
-      return FA_ERR_CUDA;
-    attr_done = true;
+  static DeviceOnce once;  // per instantiation: attributes set on each device used
+  {
+    const int rc_once = once_per_device(once, [&]() -> int {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes) != cudaSuccess)
+        return int(FA_ERR_CUDA);
+      // the kernel moves registers between warpgroups (setmaxnreg); that is only
+      // sound when it is launched with exactly the planned count per thread
+      cudaFuncAttributes fattr{};
+      if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess || fattr.numRegs != Cfg::kRegsLaunch)
+        return int(FA_ERR_CUDA);
+      return int(FA_OK);
+    });
+    if (rc_once) return rc_once;
   }
   dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
@@ -188,12 +210,15 @@ int launch_fwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMa
                   const fa::FwdParams& prm, cudaStream_t st) {
   using Cfg = fa::Fwd256Cfg;
   auto kern = fa::fa_fwd256_kernel<BF16>;
-  static bool attr_done = false;  // per instantiation and process
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
-      return FA_ERR_CUDA;
-    attr_done = true;
+  static DeviceOnce once;  // per instantiation: attributes set on each device used
+  {
+    const int rc_once = once_per_device(once, [&]() -> int {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes) != cudaSuccess)
+        return int(FA_ERR_CUDA);
+      return int(FA_OK);
+    });
+    if (rc_once) return rc_once;
   }
   dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
@@ -224,17 +249,20 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   if (rc) return rc;
   using Cfg = fa::BwdCfg<D>;
   auto kern = fa::fa_bwd_main_kernel<D, BF16, DROP>;
-  static bool attr_done = false;  // per instantiation and process
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
-      return FA_ERR_CUDA;
-    // the kernel moves registers between warpgroups (setmaxnreg); that is only
-    // sound when it is launched with exactly the planned count per thread
-    cudaFuncAttributes fattr{};
-    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess || fattr.numRegs != Cfg::kRegsLaunch)
-      return FA_ERR_CUDA;
-    attr_done = true;
+  static DeviceOnce once;  // per instantiation: attributes set on each device used
+  {
+    const int rc_once = once_per_device(once, [&]() -> int {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes) != cudaSuccess)
+        return int(FA_ERR_CUDA);
+      // the kernel moves registers between warpgroups (setmaxnreg); that is only
+      // sound when it is launched with exactly the planned count per thread
+      cudaFuncAttributes fattr{};
+      if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess || fattr.numRegs != Cfg::kRegsLaunch)
+        return int(FA_ERR_CUDA);
+      return int(FA_OK);
+    });
+    if (rc_once) return rc_once;
   }
   dim3 grid(unsigned(prm.B * prm.Hkv), unsigned(prm.n_ntiles));
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, prm);
@@ -273,9 +301,7 @@ int fa_set_bwd_main_events(void* ev_start, void* ev_stop) {
 }
 
 uint64_t fa_set_wait_limit_ns(uint64_t limit_ns) {
-  const uint64_t old = g_wait_limit_ns;
-  g_wait_limit_ns = limit_ns;
-  return old;
+  return g_wait_limit_ns.exchange(limit_ns, std::memory_order_relaxed);
 }
 
 }  // extern "C"
@@ -328,7 +354,7 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   prm.wl = window_left;
   prm.wr = window_right;
   prm.err = device_error_ptr();
-  prm.wait_limit_ns = g_wait_limit_ns;
+  prm.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   prm.cu_q = cu_q;
   prm.cu_k = cu_k;
   prm.total_q = total_q;
@@ -524,7 +550,7 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   bp.wl = window_left;
   bp.wr = window_right;
   bp.err = err;
-  bp.wait_limit_ns = g_wait_limit_ns;
+  bp.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   bp.cu_q = cu_q;
   bp.cu_k = cu_k;
   bp.total_q = total_q;
@@ -656,25 +682,19 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kNoAllocMaxDevices = 64;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
-std::mutex g_noalloc_mutex;
-
-// Device address of the scratch array on the current device (looked up on the
-// first call per device), or nullptr on failure.
+// Device address of the scratch array on the current device, or nullptr on
+// failure.  It is looked up on every call (cheap once the module is loaded on
+// the device), so a context that was torn down and created again is never
+// handed a stale address.
 void* noalloc_scratch_address() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_addr[dev] = p;
-  }
-  return g_noalloc_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace
+
+extern "C" size_t fa_bwd_noalloc_scratch_bytes(void) { return FA_BWD_NOALLOC_SCRATCH_BYTES; }
 
 extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
@@ -701,17 +721,14 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
 namespace {
 
 int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      n = v;
-    else
-      n = 148;
-  });
-  return n;
+  static std::atomic<int> cached[kMaxDevices];  // 0 = not yet read
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < kMaxDevices && (v = cached[dev].load(std::memory_order_relaxed)) > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    return 148;
+  if (dev < kMaxDevices) cached[dev].store(v, std::memory_order_relaxed);
+  return v;
 }
 
 // Splits of the key tiles of every (sequence, kv head): enough CTAs for about
@@ -807,12 +824,15 @@ int launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMa
                   const fa::DecodeParams& prm, cudaStream_t st) {
   using Cfg = fa::DecCfg<D>;
   auto kern = fa::fa_decode_kernel<D, BF16>;
-  static bool attr_done = false;  // per instantiation and process
-  if (!attr_done) {  // room for the largest query tile (128 rows)
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::smem_bytes(128)) != cudaSuccess)
-      return FA_ERR_CUDA;
-    attr_done = true;
+  static DeviceOnce once;  // per instantiation: attributes set on each device used
+  {
+    const int rc_once = once_per_device(once, [&]() -> int {  // room for the largest query tile (128 rows)
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::smem_bytes(128)) != cudaSuccess)
+        return int(FA_ERR_CUDA);
+      return int(FA_OK);
+    });
+    if (rc_once) return rc_once;
   }
   const int smem = Cfg::smem_bytes((prm.R + 7) & ~7);
   dim3 grid(unsigned(prm.n_splits), unsigned(prm.Hkv), unsigned(prm.B));
@@ -929,7 +949,7 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
                                              ((rows * d * sizeof(float) + 255) & ~size_t(255)));
   }
   prm.err = device_error_ptr();
-  prm.wait_limit_ns = g_wait_limit_ns;
+  prm.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   if (!prm.err) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16)
@@ -986,12 +1006,15 @@ int launch_fwd_fp8(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
                    const fa::Fp8Params& prm, cudaStream_t st) {
   using Cfg = fa::Fp8Cfg<D>;
   auto kern = fa::fa_fwd_fp8_kernel<D>;
-  static bool attr_done = false;  // per instantiation and process
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
-      return FA_ERR_CUDA;
-    attr_done = true;
+  static DeviceOnce once;  // per instantiation: attributes set on each device used
+  {
+    const int rc_once = once_per_device(once, [&]() -> int {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes) != cudaSuccess)
+        return int(FA_ERR_CUDA);
+      return int(FA_OK);
+    });
+    if (rc_once) return rc_once;
   }
   dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
@@ -1058,7 +1081,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.wl = window_left;
   prm.wr = window_right;
   prm.err = device_error_ptr();
-  prm.wait_limit_ns = g_wait_limit_ns;
+  prm.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   if (!prm.err) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_fwd_fp8<64>(mq, mk, mv, prm, st)

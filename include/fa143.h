@@ -231,8 +231,10 @@ size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d);
  *   dq         [B, Nq, Hq, d]  written
  *   dk, dv     [B, Nk, Hkv, d] written
  *   workspace  >= fa_bwd_workspace_size(B, Nq, Hq, d) bytes, device memory
- * Launches a short sequence of kernels on `stream`.  dQ is accumulated with
- * fp32 atomics, so its last bits may differ from run to run.
+ * Launches a short sequence of kernels on `stream`.  The partial dQ of the
+ * key tiles are added into the fp32 accumulator with bulk tensor reduce-adds
+ * in an order that varies from run to run, so dQ's last bits may differ
+ * between runs; dK and dV are summed without atomics and are reproducible.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
            const float* lse, void* dq, void* dk, void* dv, void* workspace,
@@ -259,16 +261,23 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
  *
  *  - Sizes whose fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_SCRATCH_BYTES
  *    are rejected with FA_ERR_WORKSPACE before anything is launched.
- *  - The first call on a device looks up the buffer's device address (once
- *    per device, with that device current); make that first call before any
- *    stream capture.
+ *  - Each call looks up the buffer's device address on the current device
+ *    (cudaGetSymbolAddress).  The first call on a device is also where the
+ *    runtime loads the library's device code there; make that first call
+ *    before any stream capture.
  *  - All calls share the one buffer, which keeps the previous call's
  *    contents (the kernels re-initialise what must start at zero).  Calls
  *    that overlap on the GPU (for example on two streams at once) race on it.
- * Results equal fa_bwd's (dQ up to the order of its fp32 atomic adds).
+ * Results equal fa_bwd's (dQ up to the order of its fp32 reduce-adds).
  * The pages describe no such variant; it has no counterpart there.
  */
 #define FA_BWD_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* The size of that built-in scratch buffer in bytes
+ * (FA_BWD_NOALLOC_SCRATCH_BYTES as the library was built), so a caller can
+ * check fa_bwd_workspace_size() against the library it actually loaded.
+ * Host only; never fails. */
+size_t fa_bwd_noalloc_scratch_bytes(void);
 
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                    const void* dout, const float* lse, void* dq, void* dk, void* dv,
