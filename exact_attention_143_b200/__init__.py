@@ -36,7 +36,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 # names exported by libfa143.so (the declarations of include/fa143.h)
 EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
-            "fa_bwd_noalloc", "fa_bwd_noalloc_scratch_bytes", "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
+            "fa_bwd_noalloc", "fa_bwd_noalloc_scratch_bytes", "fa_selftest_wait_timeout", "fa_selftest_exp2", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_fwd_paged_workspace_size", "fa_fwd_paged", "fa_fwd_fp8", "fa_fwd_dropout",
             "fa_bwd_dropout")
 
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_set_bwd_main_events.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [i64p] * 8 + [i, f, i, i, i, vp]
     lib.fa_bwd_noalloc.restype = i
+    lib.fa_selftest_exp2.argtypes = [vp, vp, i, i, vp]
+    lib.fa_selftest_exp2.restype = i
     lib.fa_bwd_noalloc_scratch_bytes.argtypes = []
     lib.fa_bwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.fa_fwd_varlen.argtypes = [vp] * 7 + [i] * 8 + [i64p] * 4 + [i, f, i, i, i, vp]
@@ -341,6 +343,22 @@ def selftest_wait_timeout(limit_ns: int, device=None) -> int:
     if rc:
         raise FAError(rc, "fa_selftest_wait_timeout")
     return get_device_error(dev)
+
+
+def selftest_exp2(x, bf16=False):
+    """2^x by the kernels' FMA-pipe polynomial, for x an fp32 CUDA tensor."""
+    lib = load_library()
+    dev = _check_cuda(x)
+    if x.dtype != torch.float32:
+        raise TypeError("x must be fp32")
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        rc = lib.fa_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), int(bool(bf16)),
+                                  _stream(dev))
+    if rc:
+        raise FAError(rc, "fa_selftest_exp2")
+    return y
 
 
 def set_wait_limit_ns(limit_ns: int) -> int:

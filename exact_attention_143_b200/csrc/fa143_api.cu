@@ -180,6 +180,17 @@ __global__ void fa_selftest_wait_kernel(unsigned int* err, uint64_t limit_ns) {
   }
 }
 
+// 2^x by the FMA-pipe polynomial the softmax uses for part of its column
+// pairs, one pair per thread, so it can be tested against the exact function.
+__global__ void fa_selftest_exp2_kernel(const float* x, float* y, int n, int bf16) {
+  const int i = 2 * int(blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 in = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 r = bf16 ? fa::exp2_fma_pair<true>(in) : fa::exp2_fma_pair<false>(in);
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
+
 template <int D, bool BF16, bool DROP = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const fa::FwdParams& prm, cudaStream_t st) {
@@ -291,6 +302,16 @@ int fa_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   unsigned int* err = device_error_ptr();
   if (!err) return FA_ERR_CUDA;
   fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_selftest_exp2(const float* x, float* y, int n, int bf16, void* stream) {
+  if (x == nullptr || y == nullptr || n < 1) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u))
+    return FA_ERR_ALIGNMENT;
+  const int pairs = (n + 1) / 2;
+  fa_selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, y, n, bf16);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

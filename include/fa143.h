@@ -338,6 +338,18 @@ int fa_set_bwd_main_events(void* ev_start, void* ev_stop);
 int fa_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /*
+ * Self-test of the FMA-pipe 2^x that the softmax uses for part of its
+ * exponentials (a degree-3 minimax polynomial for 2^f on [-1/2, 1/2] times
+ * 2^n built in the exponent bits; x is clamped at -127, where the result is
+ * +0).  Writes y[i] = that 2^x[i] for i < n (x, y: device fp32, 4-byte
+ * aligned); bf16 != 0 selects the instantiation the bf16 kernels use.  One
+ * launch on `stream`.  Returns FA_ERR_INVALID_ARG for null pointers or n < 1,
+ * FA_ERR_ALIGNMENT for misaligned pointers.  The pages have no counterpart:
+ * it exists so the approximation can be checked against the exact function.
+ */
+int fa_selftest_exp2(const float* x, float* y, int n, int bf16, void* stream);
+
+/*
  * Sets the per-wait limit of device-side waits, in nanoseconds (default
  * 2e9).  Returns the previous value.  For tests of the timeout path only.
  */

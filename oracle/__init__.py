@@ -93,6 +93,9 @@ class Oracle:
         lib.oracle_dropout_keep.restype = i
         lib.oracle_fwd_dropout.argtypes = [dp, dp, dp, dp, dp] + shape + [i, u64, u32, i]
         lib.oracle_fwd_dropout.restype = i
+        lib.oracle_fwd_rows_dropout.argtypes = ([dp, dp, dp, ip, ctypes.c_long, dp, dp] + shape +
+                                                [i, u64, u32, i])
+        lib.oracle_fwd_rows_dropout.restype = i
         lib.oracle_bwd_dropout.argtypes = [dp] * 9 + shape + [i, u64, u32, i]
         lib.oracle_bwd_dropout.restype = i
         lib.oracle_default_threads.argtypes = []
@@ -204,6 +207,24 @@ class Oracle:
             raise RuntimeError("oracle_fwd_dropout failed")
         return o, lse
 
+    def attention_fwd_rows_dropout(self, q, k, v, rows, softmax_scale, keep_T, seed, offset,
+                                   causal=False, window_size=(-1, -1), nthreads=0):
+        """O [n,d] and LSE [n] with dropout for selected rows (b, h, i)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        n = rows.shape[0]
+        o = np.zeros((n, d), np.float64)
+        lse = np.zeros((n,), np.float64)
+        c, wl, wr = _mask_args(causal, window_size)
+        rc = self.lib.oracle_fwd_rows_dropout(
+            _ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n,
+            _ptr(o), _ptr(lse), B, Nq, Nk, Hq, Hkv, d, float(softmax_scale), c, wl, wr,
+            int(keep_T), int(seed), int(offset), int(nthreads))
+        if rc:
+            raise RuntimeError("oracle_fwd_rows_dropout failed")
+        return o, lse
+
     def attention_bwd_dropout(self, q, k, v, dout, softmax_scale, keep_T, seed, offset,
                               causal=False, window_size=(-1, -1), nthreads=0):
         """dQ, dK, dV, LSE and D with dropout at keep threshold keep_T."""
@@ -276,6 +297,10 @@ def attention_fwd_paged(*a, **kw):
 
 def attention_fwd_dropout(*a, **kw):
     return _get().attention_fwd_dropout(*a, **kw)
+
+
+def attention_fwd_rows_dropout(*a, **kw):
+    return _get().attention_fwd_rows_dropout(*a, **kw)
 
 
 def attention_bwd_dropout(*a, **kw):

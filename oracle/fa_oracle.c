@@ -494,6 +494,25 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
 }
 
 /* The forward and backward with dropout at keep threshold T (1..255). */
+/* Selected rows of the forward with dropout (rows as in oracle_fwd_rows):
+ * the same per-row definition, for checking long sequences one row at a time. */
+int oracle_fwd_rows_dropout(const double* q, const double* k, const double* v,
+                            const int64_t* rows, long nrows, double* o_rows, double* lse_rows,
+                            int B, int Nq, int Nk, int Hq, int Hkv, int d, double tau, int causal,
+                            int window_left, int window_right, int T, uint64_t seed,
+                            uint32_t offset, int nthreads) {
+    if (T < 1 || T > 255) return -1;
+    fwd_ctx c = {{B, Nq, Nk, Hq, Hkv, d, tau, causal, window_left, window_right, T, seed, offset},
+                 q, k, v, o_rows, lse_rows, rows};
+    if (check_shape(&c.s)) return -1;
+    for (long r = 0; r < nrows; ++r) {
+        if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 || rows[3 * r + 1] >= Hq ||
+            rows[3 * r + 2] < 0 || rows[3 * r + 2] >= Nq)
+            return -1;
+    }
+    return run_pool(fwd_rows_item, &c, nrows, 2 * (size_t)Nk, nthreads);
+}
+
 int oracle_fwd_dropout(const double* q, const double* k, const double* v, double* o, double* lse,
                        int B, int Nq, int Nk, int Hq, int Hkv, int d, double tau, int causal,
                        int window_left, int window_right, int T, uint64_t seed, uint32_t offset,

@@ -11,7 +11,7 @@ import torch
 
 import exact_attention_143_b200 as fa
 import oracle
-from seeded_inputs import make_qkv
+from seeded_inputs import WORKLOADS, make_qkv, make_workload_inputs, sample_rows
 from tests.parity import check_grad, check_lse, check_o, to64
 
 pytestmark = pytest.mark.gpu
@@ -75,3 +75,30 @@ def test_dropout_rejects_p_near_one():
     with pytest.raises(fa.FAError) as e:
         fa.fa_fwd(q, k, v, dropout_p=0.999)
     assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+def test_dropout_full_size_rows_past_8192():
+    # the benchmark's dropout workload (16384 tokens, 16 heads, d 128, bf16,
+    # causal, p = 0.1): rows above 2^13 and keys up to 16383 exercise the
+    # high bits of the generator's row and column counters, which the small
+    # cases above never reach
+    w = WORKLOADS["fwdbwd_1x16384_h16_d128_bf16_causal"]
+    q, k, v = make_workload_inputs(w, with_dout=False)
+    p, seed, offset = 0.1, 1234, 0
+    o, lse = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), softmax_scale=w.softmax_scale,
+                       causal=True, dropout_p=p, seed=seed, offset=offset)
+    torch.cuda.synchronize()
+    assert fa.get_device_error() == fa.FA_OK
+    rows = sample_rows(w.batch, w.q_heads, w.seqlen_q, 48, w.seed + 100)
+    extra = np.array([[0, h, i] for h, i in ((0, 8191), (1, 8192), (5, 12345), (15, 16383),
+                                             (7, 16256), (9, 10240))])
+    rows = np.unique(np.concatenate([rows, extra]), axis=0)
+    assert (rows[:, 2] > 8192).sum() >= 20
+    T = oracle.dropout_keep_threshold(p)
+    o_ref, lse_ref = oracle.attention_fwd_rows_dropout(to64(q), to64(k), to64(v), rows,
+                                                       w.softmax_scale, T, seed, offset, True)
+    o_cpu, lse_cpu = o.cpu(), lse.cpu()
+    o_rows = np.stack([to64(o_cpu[b, i, h]) for b, h, i in rows])
+    lse_rows = np.array([float(lse_cpu[b, h, i]) for b, h, i in rows])
+    check_o(o_rows, o_ref, w.dtype)
+    check_lse(lse_rows, lse_ref)

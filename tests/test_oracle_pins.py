@@ -502,6 +502,21 @@ def test_rows_subset_matches_full(orc):
         orc.attention_fwd_rows(q, k, v, np.array([[0, 0, 33]]), 0.25)
 
 
+def test_rows_dropout_subset_matches_full(orc):
+    # the row-at-a-time dropout forward picks the same rows, keep bits and
+    # rescaling as the full dropout forward (pinned by check_dropout)
+    q, k, v = rand((2, 45, 4, 16), 95), rand((2, 50, 2, 16), 96), rand((2, 50, 2, 16), 97)
+    T, seed, offset = 200, 0x1234ABCD, 3
+    o, lse = orc.attention_fwd_dropout(q, k, v, 0.3, T, seed, offset, True, (7, -1))
+    rows = np.array([[0, 0, 0], [1, 3, 44], [0, 2, 17], [1, 1, 5]])
+    orow, lrow = orc.attention_fwd_rows_dropout(q, k, v, rows, 0.3, T, seed, offset, True, (7, -1))
+    for r, (b, h, i) in enumerate(rows):
+        np.testing.assert_array_equal(orow[r], o[b, i, h])
+        assert lrow[r] == lse[b, h, i]
+    with pytest.raises(RuntimeError):
+        orc.attention_fwd_rows_dropout(q, k, v, rows, 0.3, 0, seed, offset)  # T out of range
+
+
 def test_thread_count_does_not_change_bits(orc):
     q, k, v, do = (rand((1, 37, 2, 8), s) for s in (101, 102, 103, 104))
     a = orc.attention_bwd(q, k, v, do, 0.3, True, nthreads=1)
