@@ -243,6 +243,60 @@ def oracle_sample_rate(w: Workload, budget_s: float):
     return flops / dt / 1e12, sample, _o.default_threads(), T, dt
 
 
+# the pages' five benchmark configurations, in order (the sixth workload, d = 256,
+# is this library's own addition)
+CONFIGS = ["tiny_128_d64_fp16", "fwd_2x2048_h8_d64_fp16", "fwd_2x2048_h8_d64_fp16_causal",
+           "fwd_4x4096_h32_d64_fp16_causal", "fwd_2x4096_h32kv8_d128_bf16_causal_win256",
+           "fwdbwd_1x16384_h16_d128_bf16_causal"]
+
+
+def oracle_config_times(budget_s: float):
+    """Wall time of the fp64 oracle on every configuration: measured on the whole
+    configuration where that fits about budget_s, otherwise on a prefix of one
+    (batch, head) and extrapolated.  The oracle materialises every score of a
+    (batch, head), so its cost is proportional to B * Hq * Nq * Nk: the full-size
+    time is the sample time times that count over the sample's T * T."""
+    import oracle
+    f = lambda t: t.float().double().numpy()  # noqa: E731
+    out = {}
+    for name in CONFIGS:
+        w = WORKLOADS[name]
+        full_units = w.batch * w.q_heads * w.seqlen_q * w.seqlen_k
+
+        def run(B, H, Hk, T, bwd):
+            q, k, v, do = make_qkv(B, T, T, H, Hk, w.head_dim, w.dtype, w.seed, with_dout=True)
+            qq, kk, vv, dd = f(q), f(k), f(v), f(do)
+            t0 = time.perf_counter()
+            oracle.attention_fwd(qq, kk, vv, w.softmax_scale, w.causal, w.window)
+            t1 = time.perf_counter()
+            tb = None
+            if bwd:
+                oracle.attention_bwd(qq, kk, vv, dd, w.softmax_scale, w.causal, w.window)
+                tb = time.perf_counter() - t1
+            return t1 - t0, tb
+
+        ent = {}
+        if full_units <= 4 * 2048 * 2048 * 8:  # the whole configuration
+            tf, tb = run(w.batch, w.q_heads, w.kv_heads, w.seqlen_q, w.backward)
+            ent = {"fwd_s": round(tf, 3), "measured": "whole configuration"}
+            if tb is not None:
+                ent["bwd_s"] = round(tb, 3)
+        else:  # a prefix of one (batch, head), then extrapolated
+            T = min(w.seqlen_q, 1024)
+            tf, tb = run(1, 1, 1, T, w.backward)
+            grow = max(1.0, math.sqrt(budget_s / max(tf + (tb or 0.0), 1e-3)))
+            T = min(w.seqlen_q, max(T, int(T * grow) // 128 * 128))
+            tf, tb = run(1, 1, 1, T, w.backward)
+            scale = full_units / float(T * T)
+            ent = {"fwd_s": round(tf * scale, 1), "measured": "first %d tokens of one (batch, head): "
+                   "fwd %.2f s%s; full size extrapolated by B*Hq*Nq*Nk / T^2 = %.0f"
+                   % (T, tf, "" if tb is None else ", bwd %.2f s" % tb, scale)}
+            if tb is not None:
+                ent["bwd_s"] = round(tb * scale, 1)
+        out[name] = ent
+    return out
+
+
 # ---------------------------------------------------------------- our arm
 def time_steps(step, K, W, flush, stream, per_step_events=None):
     """Run W warm-up steps, then K steps each bracketed by its own events, with
@@ -506,7 +560,8 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, sample, cores, _, _ = oracle_sample_rate(w, args.cpu_seconds)
-        cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample,
+               "wall_s_per_config": oracle_config_times(args.cpu_seconds / 5.0)}
 
     if rank == 0:
         line = {
