@@ -47,29 +47,52 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return make_uint4(c0, c1, c2, c3);
 }
 
-__device__ __forceinline__ uint32_t word_of(const uint4& w, int k) {
-  return k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
+// 4 x 4 transpose across the four lanes of a group (lanes 4t .. 4t + 3): lane
+// q holds r[k] = v(q, k) on entry and v(k, q) on exit.  Two exchange rounds
+// (lane distance 1, then 2) with predicated selects: no lane-dependent
+// indexing, so no divergent branches.
+__device__ __forceinline__ void transpose4_lanes(uint32_t (&r)[4], int q) {
+  const bool o1 = (q & 1) != 0, o2 = (q & 2) != 0;
+  // round 1: entries k with bit 0 of k != bit 0 of q come from lane q ^ 1
+  uint32_t sa = o1 ? r[0] : r[1], sb = o1 ? r[2] : r[3];
+  sa = __shfl_xor_sync(0xffffffffu, sa, 1);
+  sb = __shfl_xor_sync(0xffffffffu, sb, 1);
+  if (o1) {
+    r[0] = sa;
+    r[2] = sb;
+  } else {
+    r[1] = sa;
+    r[3] = sb;
+  }
+  // round 2: entries k with bit 1 of k != bit 1 of q come from lane q ^ 2
+  sa = o2 ? r[0] : r[2];
+  sb = o2 ? r[1] : r[3];
+  sa = __shfl_xor_sync(0xffffffffu, sa, 2);
+  sb = __shfl_xor_sync(0xffffffffu, sb, 2);
+  if (o2) {
+    r[0] = sa;
+    r[1] = sb;
+  } else {
+    r[2] = sa;
+    r[3] = sb;
+  }
 }
 
 // Forward, four key groups at a time: word (i mod 4) of the generator output
 // of groups jg0/4 + 4k .. + 3 (keys jg0 + 16k .. + 15), out[m] for group 4k + m.
-// The four lanes of a 4-row group each make one of the four calls and pass
-// the words to their rows in four shuffle rounds.
+// The four lanes of a 4-row group (rows i with i mod 4 = lane mod 4) each make
+// one of the four calls; a transpose across the group hands lane q word q of
+// every call.
 __device__ __forceinline__ void dropout_row_words4(const DropoutParams& dp, uint32_t bh, int i,
                                                    int jg0, int k, uint32_t (&out)[4]) {
-  const int lane = threadIdx.x & 31, q = lane & 3;
-  const int base = lane & ~3;
+  const int q = threadIdx.x & 3;
   const uint4 w = philox4x32_10(uint32_t((jg0 >> 2) + 4 * k + q), uint32_t(i >> 2), bh, dp.offset,
                                 dp.seed_lo, dp.seed_hi);
-  uint32_t got[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t)
-    got[t] = __shfl_sync(0xffffffffu, word_of(w, (q + t) & 3), base | ((q - t) & 3));
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int t = (q - m) & 3;
-    out[m] = t == 0 ? got[0] : (t == 1 ? got[1] : (t == 2 ? got[2] : got[3]));
-  }
+  out[0] = w.x;
+  out[1] = w.y;
+  out[2] = w.z;
+  out[3] = w.w;
+  transpose4_lanes(out, q);
 }
 
 // 0xFF in each byte of `word` that is below T (T in 1..255), 0x00 elsewhere.
@@ -86,30 +109,26 @@ __device__ __forceinline__ uint32_t pair_mask(uint32_t m, int b) {
 // Backward: the keep bytes of key row j for 16 query groups (64 queries)
 // starting at query ig0 (a multiple of 4): out[g] holds, in byte k, the byte
 // of query ig0 + 4g + k, i.e. byte (j mod 4) of word k of group g's output.
-// Lanes 4t .. 4t + 3 (keys with the same j / 4) share the calls as above.
+// Lanes 4t .. 4t + 3 (keys with the same j / 4, j mod 4 = lane mod 4) share
+// the calls: lane q calls for query group 4k + q and packs, for each lane r
+// of the group, byte r of the four words; the transpose then hands lane q
+// the packs meant for it.
 __device__ __forceinline__ void dropout_col_words(const DropoutParams& dp, uint32_t bh, int j,
                                                   int ig0, uint32_t (&out)[16]) {
-  const int lane = threadIdx.x & 31, q = lane & 3;
-  const int base = lane & ~3;
+  const int q = threadIdx.x & 3;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const uint4 w = philox4x32_10(uint32_t(j >> 2), uint32_t((ig0 >> 2) + 4 * k + q), bh,
                                   dp.offset, dp.seed_lo, dp.seed_hi);
-    uint32_t got[4];
+    uint32_t pk[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      // for receiver lane r = (q + t) mod 4: byte r of each of the four words
-      const int r = (q + t) & 3;
-      const uint32_t b0 = (w.x >> (8 * r)) & 0xFFu, b1 = (w.y >> (8 * r)) & 0xFFu;
-      const uint32_t b2 = (w.z >> (8 * r)) & 0xFFu, b3 = (w.w >> (8 * r)) & 0xFFu;
-      const uint32_t packed = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-      got[t] = __shfl_sync(0xffffffffu, packed, base | ((q - t) & 3));
-    }
+    for (int r = 0; r < 4; ++r)  // byte r of each of the four words
+      pk[r] = __byte_perm(__byte_perm(w.x, w.y, 0x40 | r | ((4 + r) << 4)),
+                          __byte_perm(w.z, w.w, 0x40 | r | ((4 + r) << 4)),
+                          0x5410);
+    transpose4_lanes(pk, q);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int t = (q - m) & 3;
-      out[4 * k + m] = t == 0 ? got[0] : (t == 1 ? got[1] : (t == 2 ? got[2] : got[3]));
-    }
+    for (int m = 0; m < 4; ++m) out[4 * k + m] = pk[m];
   }
 }
 
