@@ -457,6 +457,23 @@ def run_ours(args):
             table[name] = {"fwd_ms_median": round(med, 4), "fwd_ms_min": round(min(tms), 4),
                            "fwd_ms_median_warm_l2": round(statistics.median(wms), 4),
                            "fwd_tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
+            if tw.head_dim == 256:
+                # the head_dim 256 backward (two halves of d per key tile),
+                # dO i.i.d. N(0, 1) like the other backward workloads
+                tdo = torch.randn(tq.shape, generator=torch.Generator().manual_seed(tw.seed + 1)
+                                  ).to(tw.dtype).to(dev)
+                fa.fa_fwd(tq, tk, tv, out=to, lse=tl, **tkw)
+                tws = torch.empty(fa.bwd_workspace_size(tw.batch, tw.seqlen_q, tw.q_heads, 256),
+                                  dtype=torch.uint8, device=dev)
+                tdq, tdk, tdv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
+                bwd1 = lambda _: fa.fa_bwd(tdo, tq, tk, tv, to, tl, dq=tdq, dk=tdk, dv=tdv,  # noqa: E731
+                                           workspace=tws, **tkw)
+                bms = time_steps(bwd1, 20, 5, flush, stream)
+                bmed = statistics.median(bms)
+                btf = 2.5 * fwd_flops(tw) / (bmed / 1e3) / 1e12
+                table[name].update({"bwd_ms_median": round(bmed, 4), "bwd_tflops": round(btf, 1),
+                                    "bwd_frac_of_peak": round(btf / peak, 4)})
+                del tdo, tws, tdq, tdk, tdv
             del tq, tk, tv, to, tl
         # packed variable-length batch (no padding): forward and backward
         for vw in VARLEN_WORKLOADS.values():

@@ -15,6 +15,7 @@
 #include "fa143.h"
 #include "fa_bwd.cuh"
 #include "fa_bwd_aux.cuh"
+#include "fa_bwd256.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd256.cuh"
@@ -239,7 +240,7 @@ int launch_fwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMa
 // 3-D fp32 tensor map over the dQ accumulator [B*Hq, Nq, d] for the bulk
 // reduce-adds: box of 32 columns (128 B, 128-byte swizzle) x rows_per_box rows.
 int make_dq_acc_map(CUtensorMap* map, float* dq_acc, int B, int Nq, int Hq, int d,
-                    int rows_per_box) {
+                    int rows_per_box, bool swizzle128 = true) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return FA_ERR_CUDA;
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(Nq), cuuint64_t(B) * cuuint64_t(Hq)};
@@ -247,7 +248,8 @@ int make_dq_acc_map(CUtensorMap* map, float* dq_acc, int B, int Nq, int Hq, int 
   cuuint32_t box[3] = {32, cuuint32_t(rows_per_box), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
@@ -276,6 +278,29 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     if (rc_once) return rc_once;
   }
   dim3 grid(unsigned(prm.B * prm.Hkv), unsigned(prm.n_ntiles));
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool BF16>
+int launch_bwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const CUtensorMap& mdo, const fa::BwdParams& prm, cudaStream_t st) {
+  using Cfg = fa::Bwd256Cfg;
+  CUtensorMap mdq;  // fp32 dQ accumulator, blocks of 32 columns x 32 rows, unswizzled
+  int rc = make_dq_acc_map(&mdq, prm.dq_acc, prm.B, prm.Nq, prm.Hq, Cfg::D, Cfg::kQ, false);
+  if (rc) return rc;
+  auto kern = fa::fa_bwd256_main_kernel<BF16>;
+  static DeviceOnce once;  // per instantiation: attributes set on each device used
+  {
+    const int rc_once = once_per_device(once, [&]() -> int {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes) != cudaSuccess)
+        return int(FA_ERR_CUDA);
+      return int(FA_OK);
+    });
+    if (rc_once) return rc_once;
+  }
+  dim3 grid(unsigned(prm.B * prm.Hkv), unsigned(prm.n_ntiles), 2u);  // z: half of d
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -502,9 +527,12 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
     if (overlaps(w0, w0 + need, l0, l0 + lse_bytes)) return FA_ERR_INVALID_ARG;
   }
 
+  if (drop && d == 256) return FA_ERR_UNSUPPORTED;
+  // d = 256 streams Q and dO in steps of 32 query rows
+  const int q_rows = d == 256 ? fa::Bwd256Cfg::kQ : 128;
   CUtensorMap mq, mk, mv, mdo;
-  if ((rc = make_map(&mq, tq, dtype)) || (rc = make_map(&mk, tk, dtype)) ||
-      (rc = make_map(&mv, tv, dtype)) || (rc = make_map(&mdo, tdo, dtype)))
+  if ((rc = make_map(&mq, tq, dtype, q_rows)) || (rc = make_map(&mk, tk, dtype)) ||
+      (rc = make_map(&mv, tv, dtype)) || (rc = make_map(&mdo, tdo, dtype, q_rows)))
     return rc;
   unsigned int* err = device_error_ptr();
   if (!err) return FA_ERR_CUDA;
@@ -578,7 +606,10 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   bp.total_k = total_k;
   if (drop) bp.drop = *drop;
   if (g_bwd_ev_start && cudaEventRecord(g_bwd_ev_start, st) != cudaSuccess) return FA_ERR_CUDA;
-  if (drop) {
+  if (d == 256) {
+    rc = bf16 ? launch_bwd256<true>(mq, mk, mv, mdo, bp, st)
+              : launch_bwd256<false>(mq, mk, mv, mdo, bp, st);
+  } else if (drop) {
     if (bf16)
       rc = d == 64 ? launch_bwd<64, true, true>(mq, mk, mv, mdo, bp, st)
                    : launch_bwd<128, true, true>(mq, mk, mv, mdo, bp, st);
@@ -630,7 +661,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            const int64_t o_stride[3], const int64_t do_stride[3], const int64_t dq_stride[3],
            const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
            float softmax_scale, int causal, int window_left, int window_right, void* stream) {
-  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
+  int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right,
+                        true);
   if (rc) return rc;
   if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
       !dk_stride || !dv_stride)
@@ -659,7 +691,7 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                   float softmax_scale, int causal, int window_left, int window_right,
                   void* stream) {
   int rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale,
-                        window_left, window_right);
+                        window_left, window_right, true);
   if (rc) return rc;
   if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
                          total_k)))

@@ -71,11 +71,12 @@ def test_d256_varlen():
         check_lse(lse[:, a:e][None], lse_ref, "LSE[seq %d]" % bi)
 
 
-def test_d256_backward_unsupported():
+def test_d256_dropout_backward_unsupported():
+    # the head_dim 256 backward has no dropout variant
     q, k, v = (t.to(DEV) for t in make_qkv(1, 64, 64, 2, 2, 256, torch.bfloat16, 74))
     o, lse = fa.fa_fwd(q, k, v)
     with pytest.raises(fa.FAError) as e:
-        fa.fa_bwd(torch.ones_like(o), q, k, v, o, lse)
+        fa.fa_bwd(torch.ones_like(o), q, k, v, o, lse, dropout_p=0.1, seed=1)
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
 
 
