@@ -38,7 +38,7 @@ EXPORTED = ("fa_status_string", "fa_fwd", "fa_bwd_workspace_size", "fa_bwd",
             "fa_get_device_error", "fa_set_wait_limit_ns", "fa_set_bwd_main_events",
             "fa_bwd_noalloc", "fa_bwd_noalloc_scratch_bytes", "fa_selftest_wait_timeout", "fa_selftest_exp2", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_fwd_paged_workspace_size", "fa_fwd_paged", "fa_fwd_fp8", "fa_fwd_dropout",
-            "fa_bwd_dropout")
+            "fa_bwd_dropout", "fa_fwd_varlen_dropout", "fa_bwd_varlen_dropout")
 
 _lib = None
 
@@ -102,6 +102,12 @@ def load_library(path: str = LIB_PATH):
     lib.fa_bwd_dropout.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [i] * 6 + [i64p] * 8 +
                                    [i, f, i, i, i, f, u64, u32, vp])
     lib.fa_bwd_dropout.restype = i
+    lib.fa_fwd_varlen_dropout.argtypes = ([vp] * 7 + [i] * 8 + [i64p] * 4 +
+                                          [i, f, i, i, i, f, u64, u32, vp])
+    lib.fa_fwd_varlen_dropout.restype = i
+    lib.fa_bwd_varlen_dropout.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [vp, vp] + [i] * 8 +
+                                          [i64p] * 8 + [i, f, i, i, i, f, u64, u32, vp])
+    lib.fa_bwd_varlen_dropout.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -202,11 +208,14 @@ def _check_cu(cu, n):
 
 
 def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                  softmax_scale=None, causal=False, window_size=(-1, -1), out=None, lse=None):
+                  softmax_scale=None, causal=False, window_size=(-1, -1), out=None, lse=None,
+                  dropout_p=0.0, seed=0, offset=0):
     """Forward over a packed variable-length batch (no padding).
 
     q [total_q, Hq, d], k/v [total_k, Hkv, d]; cu_seqlens_q/k int32 [B+1] on the
-    device.  Returns (o [total_q, Hq, d], lse [Hq, total_q] fp32)."""
+    device.  Returns (o [total_q, Hq, d], lse [Hq, total_q] fp32).  With
+    dropout_p > 0 the keep bits of sequence b are those a dense batch draws for
+    batch index b, at positions counted from the start of the sequence."""
     lib = load_library()
     dev = _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
     code = _dtype_code(q)
@@ -222,22 +231,29 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_
     if lse is None:
         lse = torch.empty((Hq, total_q), dtype=torch.float32, device=dev)
     wl, wr = window_size
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+            int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, _strides2(q), _strides2(k),
+            _strides2(v), _strides2(out), code, _scale(softmax_scale, d), int(bool(causal)),
+            int(wl), int(wr))
     with torch.cuda.device(dev):
-        rc = lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                               lse.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
-                               B, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, Hq,
-                               Hkv, d, _strides2(q), _strides2(k), _strides2(v), _strides2(out),
-                               code, _scale(softmax_scale, d), int(bool(causal)), int(wl),
-                               int(wr), _stream(dev))
+        if dropout_p:
+            name = "fa_fwd_varlen_dropout"
+            rc = lib.fa_fwd_varlen_dropout(*args, float(dropout_p), int(seed), int(offset),
+                                           _stream(dev))
+        else:
+            name = "fa_fwd_varlen"
+            rc = lib.fa_fwd_varlen(*args, _stream(dev))
     if rc:
-        raise FAError(rc, "fa_fwd_varlen")
+        raise FAError(rc, name)
     return out, lse
 
 
 def fa_bwd_varlen(dout, q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                   max_seqlen_k, softmax_scale=None, causal=False, window_size=(-1, -1),
-                  dq=None, dk=None, dv=None, workspace=None):
-    """Backward over a packed variable-length batch; returns (dq, dk, dv)."""
+                  dq=None, dk=None, dv=None, workspace=None, dropout_p=0.0, seed=0, offset=0):
+    """Backward over a packed variable-length batch; returns (dq, dk, dv).  dropout_p,
+    seed and offset must be those given to the forward."""
     lib = load_library()
     dev = _check_cuda(dout, q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k)
     code = _dtype_code(q)
@@ -259,19 +275,23 @@ def fa_bwd_varlen(dout, q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_
                                 device=dev)
     _check_cuda(q, dq, dk, dv, workspace)
     wl, wr = window_size
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), cu_seqlens_q.data_ptr(),
+            cu_seqlens_k.data_ptr(), B, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k,
+            Hq, Hkv, d, _strides2(q), _strides2(k), _strides2(v), _strides2(o), _strides2(dout),
+            _strides2(dq), _strides2(dk), _strides2(dv), code, _scale(softmax_scale, d),
+            int(bool(causal)), int(wl), int(wr))
     with torch.cuda.device(dev):
-        rc = lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                               dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                               dv.data_ptr(), workspace.data_ptr(),
-                               workspace.numel() * workspace.element_size(),
-                               cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B,
-                               int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, Hq, Hkv, d,
-                               _strides2(q), _strides2(k), _strides2(v), _strides2(o),
-                               _strides2(dout), _strides2(dq), _strides2(dk), _strides2(dv),
-                               code, _scale(softmax_scale, d), int(bool(causal)), int(wl),
-                               int(wr), _stream(dev))
+        if dropout_p:
+            name = "fa_bwd_varlen_dropout"
+            rc = lib.fa_bwd_varlen_dropout(*args, float(dropout_p), int(seed), int(offset),
+                                           _stream(dev))
+        else:
+            name = "fa_bwd_varlen"
+            rc = lib.fa_bwd_varlen(*args, _stream(dev))
     if rc:
-        raise FAError(rc, "fa_bwd_varlen")
+        raise FAError(rc, name)
     return dq, dk, dv
 
 

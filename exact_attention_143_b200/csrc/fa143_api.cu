@@ -409,7 +409,7 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   if (!prm.err) return FA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (drop) {
-    if (d == 256 || cu_q) return FA_ERR_UNSUPPORTED;
+    if (d == 256) return FA_ERR_UNSUPPORTED;
     if (dtype == FA_BF16)
       return d == 64 ? launch_fwd<64, true, true>(mq, mk, mv, prm, st)
                      : launch_fwd<128, true, true>(mq, mk, mv, prm, st);
@@ -500,7 +500,6 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
              float softmax_scale, int causal, int window_left, int window_right, void* stream,
              const fa::DropoutParams* drop = nullptr) {
   int rc;
-  if (drop && cu_q) return FA_ERR_UNSUPPORTED;
   for (const TensorDesc* t : {&tq, &tk, &tv, &to, &tdo, &tdq, &tdk, &tdv})
     if ((rc = check_tensor(*t))) return rc;
   if (!lse) return FA_ERR_INVALID_ARG;
@@ -1229,6 +1228,84 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
   return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(B) * Hq * Nq * sizeof(float),
                   workspace, workspace_bytes, B, Nq, Nk, Hq, Hkv, d, nullptr, nullptr, 0, 0,
                   dtype, softmax_scale, causal, window_left, window_right, stream, &dp);
+}
+
+int fa_fwd_varlen_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                          int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq,
+                          int Hkv, int d, const int64_t q_stride[2], const int64_t k_stride[2],
+                          const int64_t v_stride[2], const int64_t o_stride[2], int dtype,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          float dropout_p, uint64_t seed, uint32_t offset, void* stream) {
+  int T = 0;
+  int rc = dropout_threshold(dropout_p, &T);
+  if (rc) return rc;
+  if (T >= 256)  // nothing is dropped
+    return fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q,
+                         max_seqlen_k, total_q, total_k, Hq, Hkv, d, q_stride, k_stride,
+                         v_stride, o_stride, dtype, softmax_scale, causal, window_left,
+                         window_right, stream);
+  rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale, window_left,
+                    window_right);
+  if (rc) return rc;
+  if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
+                         total_k)))
+    return rc;
+  if (total_q > (1 << 28) || total_k > (1 << 28)) return FA_ERR_INVALID_ARG;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, 0, q_stride[0], q_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tk{k, 0, k_stride[0], k_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc tv{v, 0, v_stride[0], v_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
+  const fa::DropoutParams dp = make_dropout(T, seed, offset);
+  return fwd_impl(tq, tk, tv, to, lse, size_t(Hq) * total_q * sizeof(float), B, max_seqlen_q,
+                  max_seqlen_k, Hq, Hkv, d, cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype,
+                  softmax_scale, causal, window_left, window_right, stream, &dp);
+}
+
+int fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, const int* cu_seqlens_q,
+                          const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
+                          int total_q, int total_k, int Hq, int Hkv, int d,
+                          const int64_t q_stride[2], const int64_t k_stride[2],
+                          const int64_t v_stride[2], const int64_t o_stride[2],
+                          const int64_t do_stride[2], const int64_t dq_stride[2],
+                          const int64_t dk_stride[2], const int64_t dv_stride[2], int dtype,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          float dropout_p, uint64_t seed, uint32_t offset, void* stream) {
+  int T = 0;
+  int rc = dropout_threshold(dropout_p, &T);
+  if (rc) return rc;
+  if (T >= 256)
+    return fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
+                         cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
+                         total_k, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride,
+                         dq_stride, dk_stride, dv_stride, dtype, softmax_scale, causal,
+                         window_left, window_right, stream);
+  rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale, window_left,
+                    window_right);
+  if (rc) return rc;
+  if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
+                         total_k)))
+    return rc;
+  if (total_q > (1 << 28) || total_k > (1 << 28)) return FA_ERR_INVALID_ARG;
+  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
+      !dk_stride || !dv_stride)
+    return FA_ERR_INVALID_ARG;
+  const TensorDesc tq{q, 0, q_stride[0], q_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tk{k, 0, k_stride[0], k_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc tv{v, 0, v_stride[0], v_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tdo{dout, 0, do_stride[0], do_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tdq{dq, 0, dq_stride[0], dq_stride[1], 1, total_q, Hq, d};
+  const TensorDesc tdk{dk, 0, dk_stride[0], dk_stride[1], 1, total_k, Hkv, d};
+  const TensorDesc tdv{dv, 0, dv_stride[0], dv_stride[1], 1, total_k, Hkv, d};
+  const fa::DropoutParams dp = make_dropout(T, seed, offset);
+  return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(Hq) * total_q * sizeof(float),
+                  workspace, workspace_bytes, B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d,
+                  cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype, softmax_scale, causal,
+                  window_left, window_right, stream, &dp);
 }
 
 }  // extern "C"

@@ -133,7 +133,10 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
  * probabilities.  The backward must get the same seed and offset.  The
  * arguments are those of fa_fwd / fa_bwd plus dropout_p in [0, 1), seed
  * and offset; T = 256 (p < 1/512) runs the plain kernels, and p so close to
- * 1 that T = 0 is FA_ERR_INVALID_ARG.  d is 64 or 128; dense batches only.
+ * 1 that T = 0 is FA_ERR_INVALID_ARG.  d is 64 or 128.  The _varlen forms take
+ * the arguments of fa_fwd_varlen / fa_bwd_varlen plus the same three; there b
+ * in the counter is the sequence index and i, j are positions within the
+ * sequence.
  */
 int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                    int Nq, int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3],
@@ -150,6 +153,24 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
                    const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
                    float softmax_scale, int causal, int window_left, int window_right,
                    float dropout_p, uint64_t seed, uint32_t offset, void* stream);
+int fa_fwd_varlen_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                          int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq,
+                          int Hkv, int d, const int64_t q_stride[2], const int64_t k_stride[2],
+                          const int64_t v_stride[2], const int64_t o_stride[2], int dtype,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          float dropout_p, uint64_t seed, uint32_t offset, void* stream);
+int fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, const int* cu_seqlens_q,
+                          const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
+                          int total_q, int total_k, int Hq, int Hkv, int d,
+                          const int64_t q_stride[2], const int64_t k_stride[2],
+                          const int64_t v_stride[2], const int64_t o_stride[2],
+                          const int64_t do_stride[2], const int64_t dq_stride[2],
+                          const int64_t dk_stride[2], const int64_t dv_stride[2], int dtype,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          float dropout_p, uint64_t seed, uint32_t offset, void* stream);
 
 /*
  * Forward on FP8 inputs: q, k, v hold float8_e4m3fn values (one byte each;

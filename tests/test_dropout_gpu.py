@@ -102,3 +102,53 @@ def test_dropout_full_size_rows_past_8192():
     lse_rows = np.array([float(lse_cpu[b, h, i]) for b, h, i in rows])
     check_o(o_rows, o_ref, w.dtype)
     check_lse(lse_rows, lse_ref)
+
+
+VARLEN_CASES = [
+    # lengths q, lengths k, Hq, Hkv, d, dtype, causal, p, seed, offset.  The
+    # causal one-token sequence has one key per row, so its exact dQ and dK
+    # vanish; p = 0.5 (multiplier 2) keeps O = 2 V exact in fp16, so D = dP
+    # holds exactly on the GPU as well (at p = 0.2 the multiplier 256 / 205
+    # rounds O, and dQ becomes rounding noise of about 1e-3 on a zero).
+    ([300, 1, 129, 64], [300, 1, 129, 64], 4, 2, 64, torch.float16, True, 0.5, 4321, 5),
+    ([130, 257, 1, 77], [200, 40, 3, 128], 4, 4, 128, torch.bfloat16, False, 0.1, 2 ** 40 + 9, 0),
+]
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=lambda c: "d%d_c%d" % (c[4], c[6]))
+def test_dropout_varlen_matches_dense_slot(case):
+    """Packed sequences with dropout.  Sequence b draws the keep bits a dense
+    batch draws at batch index b with positions counted from the start of the
+    sequence, so the oracle runs a dense batch of b + 1 slots whose slot b
+    holds sequence b (the others are zeros) and slot b is compared."""
+    lq, lk, Hq, Hkv, d, dtype, causal, p, seed, offset = case
+    seqs = [make_qkv(1, nq, nk, Hq, Hkv, d, dtype, 90 + b, with_dout=True)
+            for b, (nq, nk) in enumerate(zip(lq, lk))]
+    q, k, v, do = (torch.cat([s[i][0] for s in seqs]) for i in range(4))
+    cu_q = torch.tensor(np.concatenate([[0], np.cumsum(lq)]), dtype=torch.int32, device=DEV)
+    cu_k = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32, device=DEV)
+    scale = d ** -0.5
+    kw = dict(softmax_scale=scale, causal=causal, dropout_p=p, seed=seed, offset=offset)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = fa.fa_fwd_varlen(qd, kd, vd, cu_q, cu_k, max(lq), max(lk), **kw)
+    dq, dk, dv = fa.fa_bwd_varlen(dod, qd, kd, vd, o, lse, cu_q, cu_k, max(lq), max(lk), **kw)
+    torch.cuda.synchronize()
+    assert fa.get_device_error() == fa.FA_OK
+    T = oracle.dropout_keep_threshold(p)
+    for b, (nq, nk) in enumerate(zip(lq, lk)):
+        def slot(t, n):
+            full = torch.zeros((b + 1, n) + tuple(t.shape[2:]), dtype=t.dtype)
+            full[b] = t[0]
+            return to64(full)
+        sq, sk, sv, sdo = seqs[b]
+        o_ref, lse_ref = oracle.attention_fwd_dropout(slot(sq, nq), slot(sk, nk), slot(sv, nk),
+                                                      scale, T, seed, offset, causal)
+        r0, r1, c0, c1 = sum(lq[:b]), sum(lq[:b + 1]), sum(lk[:b]), sum(lk[:b + 1])
+        check_o(o[r0:r1], o_ref[b], dtype, "O of sequence %d" % b)
+        check_lse(lse[:, r0:r1], lse_ref[b], "LSE of sequence %d" % b)
+        gq, gk, gv, _, _ = oracle.attention_bwd_dropout(slot(sq, nq), slot(sk, nk), slot(sv, nk),
+                                                        slot(sdo, nq), scale, T, seed, offset,
+                                                        causal)
+        check_grad(dq[r0:r1], gq[b], "dQ of sequence %d" % b)
+        check_grad(dk[c0:c1], gk[b], "dK of sequence %d" % b)
+        check_grad(dv[c0:c1], gv[b], "dV of sequence %d" % b)
