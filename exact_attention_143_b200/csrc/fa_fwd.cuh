@@ -83,11 +83,14 @@ struct FwdCfg {
   static constexpr int kRegsLaunch = 168;
   static constexpr int kRegsSoftmax = D == 64 ? 216 : 200;
   static constexpr int kRegsCtl = D == 64 ? 72 : 104;  // d = 128: one warp issues every MMA
-  // Q buffers: two at d = 64, so the next work tile's Q lands while the
-  // current one is still being multiplied; one at d = 128 (shared memory)
-  static constexpr int kQBufs = D == 64 ? 2 : 1;
+  // Q slots of one 128-row tile each, used in turn (work tile i takes slots
+  // 2i and 2i + 1 modulo kQSlots) and released as soon as the last Q_t K^T of
+  // their tile is done: at d = 128 the third slot lets the next work tile's
+  // first Q tile land while both tiles of the current one are in use, and the
+  // second follows once the current Q_0 is done
+  static constexpr int kQSlots = D == 64 ? 4 : 3;
   static constexpr int kSmemQ = 1024;
-  static constexpr int kSmemK = kSmemQ + kQBufs * kTiles * kTileBytes;
+  static constexpr int kSmemK = kSmemQ + kQSlots * kTileBytes;
   static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
   static constexpr int kSmemBytes = kSmemV + kStages * kTileBytes + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
@@ -253,9 +256,9 @@ __global__ void __launch_bounds__(384, 1)
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int S = Cfg::kStages;
-  constexpr int QB = Cfg::kQBufs;
+  constexpr int NQ = Cfg::kQSlots;
   constexpr bool kRing = Cfg::kRing;
-  static_assert(S <= 4 && QB <= 2, "barrier block layout");
+  static_assert(S <= 4 && NQ <= 4, "barrier block layout");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms.
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -265,8 +268,8 @@ __global__ void __launch_bounds__(384, 1)
   // barrier block at the head of shared memory
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
-  auto bar_qfull = [&](int q) { return bar(1 + q); };    // Q buffer q landed
-  auto bar_qempty = [&](int q) { return bar(3 + q); };   // its tile's Q K^T done
+  auto bar_qfull = [&](int q) { return bar(46 + q); };   // Q slot q landed
+  auto bar_qempty = [&](int q) { return bar(50 + q); };  // its tile's Q K^T all done
   auto bar_wfull = [&](int e) { return bar(5 + e); };    // work queue entry e written
   auto bar_wempty = [&](int e) { return bar(7 + e); };   // entry e read by every role
   const uint32_t bar_clc = bar(9);                       // launch-control response
@@ -299,7 +302,7 @@ __global__ void __launch_bounds__(384, 1)
   WaitCtx wc{abort_flag, p.err, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
-    for (int q = 0; q < QB; ++q) {
+    for (int q = 0; q < NQ; ++q) {
       mbar_init(bar_qfull(q), 1);
       mbar_init(bar_qempty(q), 1);
     }
@@ -411,14 +414,16 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(bar_want);
           continue;
         }
-        const int qb = iq % QB, qu = iq / QB;
-        if (qu > 0 && !(ok = mbar_wait(bar_qempty(qb), (qu - 1) & 1, wc))) break;
-        mbar_arrive_expect_tx(bar_qfull(qb), 2 * Cfg::kTileBytes);
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2 && ok; ++t) {
+          const int sl = (2 * iq + t) % NQ, u = (2 * iq + t) / NQ;
+          if (u > 0 && !(ok = mbar_wait(bar_qempty(sl), (u - 1) & 1, wc))) break;
+          mbar_arrive_expect_tx(bar_qfull(sl), Cfg::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sbase + Cfg::kSmemQ + (qb * 2 + t) * Cfg::kTileBytes + c * Cfg::kChunk,
-                        &tmQ, bar_qfull(qb), c * 64, w.qstart + w.mblock * p.mrows + t * 128,
-                        w.h, w.bc);
+            tma_load_4d(sbase + Cfg::kSmemQ + sl * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ,
+                        bar_qfull(sl), c * 64, w.qstart + w.mblock * p.mrows + t * 128, w.h,
+                        w.bc);
+        }
+        if (!ok) break;
         for (int j = w.JLO; j < w.JHI; ++j, ++gkv) {
           if (j == w.JHI - 1) mbar_arrive(bar_want);
           const int s = gkv % S, u = gkv / S;
@@ -452,9 +457,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t dQ0 = sdesc_at(kDescK, sbase + Cfg::kSmemQ);
     const uint64_t dK0 = sdesc_at(kDescK, sbase + Cfg::kSmemK);
     const uint64_t dV0 = sdesc_at(kDescMN, sbase + Cfg::kSmemV);
-    // S = Q_t K^T of Q buffer qb into tensor-memory column `col`, K/V stage s
-    auto issue_s = [&](uint32_t col, int qb, int t, int s, uint32_t done_bar) {
-      const uint64_t qa = dQ0 + uint64_t(((qb * 2 + t) * Cfg::kTileBytes) >> 4);
+    // S = Q K^T of the Q tile in slot sl into tensor-memory column `col`, K/V stage s
+    auto issue_s = [&](uint32_t col, int sl, int s, uint32_t done_bar) {
+      const uint64_t qa = dQ0 + uint64_t((sl * Cfg::kTileBytes) >> 4);
       const uint64_t kb = dK0 + uint64_t((s * Cfg::kTileBytes) >> 4);
       if (elect_one()) {
 #pragma unroll
@@ -477,6 +482,16 @@ __global__ void __launch_bounds__(384, 1)
       }
     };
     bool ok = true;
+    // Q slots of work tile iq: each query tile's slot is awaited before its
+    // first Q K^T and released after its last (at once if it has none)
+    auto q_slot = [&](int iq, int t) { return (2 * iq + t) % NQ; };
+    auto q_wait = [&](int iq, int t) {
+      return wait_all(bar_qfull(q_slot(iq, t)), ((2 * iq + t) / NQ) & 1);
+    };
+    auto q_release = [&](int iq, int t) {
+      if (elect_one()) mma_commit(bar_qempty(q_slot(iq, t)));
+      __syncwarp();
+    };
     if constexpr (!kRing) {
       // d = 128, warp 8: P_t overlays S_t, so one warp issues everything and
       // S_t(j+1) follows P_t V_j in the in-order tensor pipe without waiting
@@ -495,12 +510,25 @@ __global__ void __launch_bounds__(384, 1)
           auto in_range = [&](int t, int j) {
             return t ? (j >= w.jlo1 && j < w.jhi1) : (j >= w.jlo0 && j < w.jhi0);
           };
-          const int qb = iq % QB;
-          if (!(ok = wait_all(bar_qfull(qb), (iq / QB) & 1))) break;
+          const int jhi[2] = {w.jhi0, w.jhi1};
+          bool qready[2] = {false, false};
+          for (int t = 0; t < 2 && ok; ++t)  // a query tile with no K tile: its slot at once
+            if (jhi[t] <= (t ? w.jlo1 : w.jlo0)) {
+              if (!(ok = q_wait(iq, t))) break;
+              q_release(iq, t);
+            }
+          if (!ok) break;
           if (!(ok = wait_all(bar_kvfull(gkv % S), (gkv / S) & 1))) break;
           tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (in_range(t, w.JLO)) issue_s(t * 128, qb, t, gkv % S, bar_sfull(t));
+          for (int t = 0; t < 2 && ok; ++t)
+            if (in_range(t, w.JLO)) {
+              if (!(ok = q_wait(iq, t))) break;
+              qready[t] = true;
+              tc_fence_after();
+              issue_s(t * 128, q_slot(iq, t), gkv % S, bar_sfull(t));
+              if (w.JLO == jhi[t] - 1) q_release(iq, t);
+            }
+          if (!ok) break;
           for (int j = w.JLO; j < w.JHI && ok; ++j, ++gkv) {
             const int s = gkv % S, s1 = (gkv + 1) % S, u1 = (gkv + 1) / S;
             bool next_ready = false;
@@ -519,8 +547,13 @@ __global__ void __launch_bounds__(384, 1)
                   if (!(ok = wait_all(bar_kvfull(s1), u1 & 1))) break;
                   next_ready = true;
                 }
+                if (!qready[t]) {
+                  if (!(ok = q_wait(iq, t))) break;
+                  qready[t] = true;
+                }
                 tc_fence_after();
-                issue_s(t * 128, qb, t, s1, bar_sfull(t));
+                issue_s(t * 128, q_slot(iq, t), s1, bar_sfull(t));
+                if (j + 1 == jhi[t] - 1) q_release(iq, t);
               }
             }
             if (!ok) break;
@@ -531,8 +564,6 @@ __global__ void __launch_bounds__(384, 1)
             __syncwarp();
           }
           if (!ok) break;
-          if (elect_one()) mma_commit(bar_qempty(qb));  // this tile's MMAs are all issued
-          __syncwarp();
           ++iq;
         }
       }
@@ -545,8 +576,11 @@ __global__ void __launch_bounds__(384, 1)
         FwdTile w;
         if (read_work(e, w) <= 0) break;
         if (!w.rows || w.JHI <= w.JLO) continue;
-        const int qb = iq % QB;
-        if (!(ok = wait_all(bar_qfull(qb), (iq / QB) & 1))) break;
+        // both Q tiles before the first Q K^T; both slots released once the
+        // tile's Q K^T are all issued (at d = 64 the four slots double-buffer
+        // whole work tiles)
+        for (int t = 0; t < 2 && ok; ++t) ok = q_wait(iq, t);
+        if (!ok) break;
         for (int j = w.JLO; j < w.JHI && ok; ++j, ++gkv) {
           const int s = gkv % S, u = gkv / S;
           bool kv_ready = false;
@@ -558,7 +592,7 @@ __global__ void __launch_bounds__(384, 1)
               if (!(ok = wait_all(bar_kvfull(s), u & 1))) break;
             }
             tc_fence_after();
-            issue_s(r * 128, qb, t, s, bar_rfull(t, r));
+            issue_s(r * 128, q_slot(iq, t), s, bar_rfull(t, r));
             if (++r == 3) {
               r = 0;
               ++ur;
@@ -569,8 +603,8 @@ __global__ void __launch_bounds__(384, 1)
           __syncwarp();
         }
         if (!ok) break;
-        if (elect_one()) mma_commit(bar_qempty(qb));  // Q buffer qb: its Q K^T all issued
-        __syncwarp();
+        q_release(iq, 0);
+        q_release(iq, 1);
         ++iq;
       }
     } else {
