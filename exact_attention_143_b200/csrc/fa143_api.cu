@@ -195,6 +195,7 @@ __global__ void fa_selftest_exp2_kernel(const float* x, float* y, int n, int bf1
 template <int D, bool BF16, bool DROP = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const fa::FwdParams& prm, cudaStream_t st) {
+  // work tiles: (batch, query head or head pair) x query blocks
   using Cfg = fa::FwdCfg<D>;
   auto kern = fa::fa_fwd_kernel<D, BF16, DROP>;
   static DeviceOnce once;  // per instantiation: attributes set on each device used
@@ -212,7 +213,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     });
     if (rc_once) return rc_once;
   }
-  dim3 grid(unsigned(prm.B * prm.Hq), unsigned(prm.n_mblocks));
+  dim3 grid(unsigned(prm.B * (prm.Hq >> prm.pair)), unsigned(prm.n_mblocks));
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -393,6 +394,17 @@ int fwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   // block sees the most keys).  The d = 256 kernel always takes 128 rows.
   prm.mrows = 256;
   if (d == 256 || (causal && int64_t(B) * Hq * ((Nq + 255) / 256) < sm_count())) prm.mrows = 128;
+  // Short key ranges (a 128-row tile sees at most 4 K tiles): a work tile
+  // takes two query heads of one GQA group over the same 128 rows, so both
+  // query tiles walk the same few K tiles side by side and share each load.
+  {
+    const int right = causal ? 0 : window_right;
+    if (d != 256 && (Hq / Hkv) % 2 == 0 && window_left >= 0 && right >= 0 &&
+        int64_t(window_left) + right <= 384) {
+      prm.pair = 1;
+      prm.mrows = 128;
+    }
+  }
   prm.n_mblocks = (Nq + prm.mrows - 1) / prm.mrows;
   prm.scale_log2 = scale_log2_of(softmax_scale);
   prm.qk_negate = softmax_scale < 0.f ? 1u : 0u;

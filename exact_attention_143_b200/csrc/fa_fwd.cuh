@@ -68,6 +68,10 @@ struct FwdParams {
   // query rows per CTA: 256 (two tiles), or 128 (tile 1 idle) where fewer
   // CTAs than SMs would otherwise run
   int mrows;
+  // 1: a work tile is the same 128 query rows of two query heads of one kv
+  // head (query tile t = head 2i + t), which then see the same K tiles; used
+  // for GQA groups with short key ranges (mrows is 128)
+  int pair;
 };
 
 template <int D>
@@ -166,8 +170,9 @@ struct FwdTile {
 // Decode the tile of block index (x, y): (batch, head) from x, query block
 // from y with the heaviest (latest, under a causal mask) blocks first.
 __device__ __forceinline__ void fwd_tile(const FwdParams& p, int x, int y, FwdTile& w) {
-  w.h = x % p.Hq;
-  w.b = x / p.Hq;
+  const int hunits = p.Hq >> p.pair;
+  w.h = (x % hunits) << p.pair;
+  w.b = x / hunits;
   w.g = w.h / (p.Hq / p.Hkv);
   w.mblock = p.n_mblocks - 1 - y;
   w.Nq = p.Nq;
@@ -188,8 +193,8 @@ __device__ __forceinline__ void fwd_tile(const FwdParams& p, int x, int y, FwdTi
   int lo[2] = {0, 0}, hi[2] = {0, 0};
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int r0 = w.mblock * p.mrows + t * 128;
-    if (t * 128 < p.mrows && r0 < w.Nq) {
+    const int r0 = w.mblock * p.mrows + (p.pair ? 0 : t * 128);
+    if ((p.pair || t * 128 < p.mrows) && r0 < w.Nq) {
       const int r1 = min(r0 + 127, w.Nq - 1);
       int lo0, hi0, lo1, hi1;
       row_key_range(r0, w.Nq, w.Nk, p.causal, p.wl, p.wr, lo0, hi0);
@@ -420,7 +425,8 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(bar_qfull(sl), Cfg::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sbase + Cfg::kSmemQ + sl * Cfg::kTileBytes + c * Cfg::kChunk, &tmQ,
-                        bar_qfull(sl), c * 64, w.qstart + w.mblock * p.mrows + t * 128, w.h,
+                        bar_qfull(sl), c * 64,
+                        w.qstart + w.mblock * p.mrows + (p.pair ? 0 : t * 128), w.h + p.pair * t,
                         w.bc);
         }
         if (!ok) break;
@@ -661,8 +667,8 @@ __global__ void __launch_bounds__(384, 1)
       FwdTile w;
       if (read_work(e, w) <= 0) break;
       if (!w.rows) continue;
-      const int b = w.b, h = w.h;
-      const int row = w.mblock * p.mrows + t * 128 + r;
+      const int b = w.b, h = w.h + p.pair * t;
+      const int row = w.mblock * p.mrows + (p.pair ? 0 : t * 128) + r;
       int lo_i, hi_i;
       row_key_range(row, w.Nq, w.Nk, p.causal, p.wl, p.wr, lo_i, hi_i);
       float m_use = -INFINITY;  // running max in scaled log2 units (reference for O and l)
@@ -838,7 +844,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool has = (n > 0) && (l > 0.f);
       const float inv_l = has ? (DROP ? p.drop.scale : 1.f) / l : 0.f;
       const float lse = has ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const bool store = row < w.Nq && t * 128 < p.mrows;  // tile 1 idles at 128 rows
+      // tile 1 idles at 128 rows unless it holds the second head
+      const bool store = row < w.Nq && (p.pair || t * 128 < p.mrows);
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + w.bc * p.o_sb +
                        int64_t(w.qstart + row) * p.o_ss + int64_t(h) * p.o_sh;
 #pragma unroll

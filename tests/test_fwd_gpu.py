@@ -67,6 +67,18 @@ def test_causal_full_grid_ragged(d, dtype, window):
     run_case(2, 300, 300, 40, 8, d, dtype, True, window, seed=9)
 
 
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)], ids=["d64", "d128"])
+@pytest.mark.parametrize("Hq,Hkv,causal,window", [
+    (8, 2, True, (200, 0)),      # G = 4, sliding window: head-pair work tiles
+    (8, 2, False, (150, 100)),   # G = 4, two-sided window
+    (16, 4, True, (384, 0)),     # G = 4, the widest window that pairs heads
+    (6, 2, True, (200, 0)),      # G = 3 (odd): one head per work tile
+], ids=["g4_causal_w200", "g4_w150_100", "g4_causal_w384", "g3_causal_w200"])
+def test_gqa_window(d, dtype, Hq, Hkv, causal, window):
+    # 700 rows: five 128-row blocks plus a ragged one
+    run_case(2, 700, 700, Hq, Hkv, d, dtype, causal, window, seed=12)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (8, 1), (6, 2)])
 def test_gqa(Hq, Hkv):
     run_case(2, 260, 260, Hq, Hkv, 128, torch.bfloat16, True, (-1, -1), seed=7)
