@@ -60,7 +60,7 @@ struct Fp8Cfg {
   static constexpr uint32_t kColO = 256;
   // shared-memory descriptor layout type: 2 = 128-byte swizzle, 4 = 64-byte
   static constexpr uint64_t kLayout = D == 128 ? 2 : 4;
-  static constexpr int kEmuPairsPer8 = D == 64 ? 3 : 0;
+  static constexpr int kEmuPairsPer8 = D == 64 ? 3 : 2;
   static constexpr float kPShift = 6.f;  // P is held as 2^6 exp2(s - m)
   static constexpr float kLazy = 2.f;    // rescale once the row max grows by more than 2^2
 };
