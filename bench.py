@@ -50,6 +50,34 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 L2_FLUSH_BYTES = 256 << 20
 
 
+# ---------------------------------------------------------------- context
+def materialised_attention(q, k, v, scale, causal, window):
+    """Standard attention with the full score matrix in memory, in plain
+    PyTorch (cuBLAS products in the input dtype, softmax in fp32): the
+    comparison the pages' speedup claims are made against ("optimizing-
+    attention-flash", Quick start; "Что такое FlashAttention…", section
+    "Основной механизм простыми словами").  Context for the bench table only;
+    the library never calls it.  q [B, Nq, Hq, d], k / v [B, Nk, Hkv, d]."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    qh = q.permute(0, 2, 1, 3)
+    kh = k.permute(0, 2, 1, 3).repeat_interleave(Hq // Hkv, dim=1)
+    vh = v.permute(0, 2, 1, 3).repeat_interleave(Hq // Hkv, dim=1)
+    scores = torch.matmul(qh, kh.transpose(2, 3)).float().mul_(scale)
+    i = torch.arange(Nq, device=q.device).view(-1, 1) + (Nk - Nq)
+    j = torch.arange(Nk, device=q.device).view(1, -1)
+    wl, wr = window
+    right = 0 if causal else wr
+    hidden = torch.zeros(Nq, Nk, dtype=torch.bool, device=q.device)
+    if right >= 0:
+        hidden |= j > i + right
+    if wl >= 0:
+        hidden |= j < i - wl
+    scores.masked_fill_(hidden, float("-inf"))
+    probs = torch.softmax(scores, dim=-1).to(q.dtype)
+    return torch.matmul(probs, vh).permute(0, 2, 1, 3)
+
+
 # ---------------------------------------------------------------- counting
 def visible_pairs(Nq, Nk, causal, window):
     """Number of (query, key) pairs the mask keeps, per (batch, head)."""
@@ -457,6 +485,14 @@ def run_ours(args):
             table[name] = {"fwd_ms_median": round(med, 4), "fwd_ms_min": round(min(tms), 4),
                            "fwd_ms_median_warm_l2": round(statistics.median(wms), 4),
                            "fwd_tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
+            # context: the materialised standard attention on the same inputs
+            std1 = lambda _: materialised_attention(tq, tk, tv, tw.softmax_scale,  # noqa: E731
+                                                    tw.causal, tw.window)
+            sms = time_steps(std1, 5, 2, flush, stream)
+            smed = statistics.median(sms)
+            table[name].update({"standard_attention_ms_median": round(smed, 4),
+                                "speedup_vs_standard": round(smed / med, 2)})
+            torch.cuda.empty_cache()
             if tw.head_dim == 256:
                 # the head_dim 256 backward (two halves of d per key tile),
                 # dO i.i.d. N(0, 1) like the other backward workloads
