@@ -35,6 +35,8 @@ CASES = [
     ([300, 1, 129, 512, 77], None, 4, 2, 128, torch.bfloat16, False, (-1, -1)),
     ([200, 333, 64], [333, 200, 64], 2, 1, 64, torch.bfloat16, True, (-1, -1)),
     ([257, 380], None, 8, 2, 128, torch.bfloat16, True, (100, 0)),
+    # head-pair work tiles (even GQA group, short window) with Nq != Nk per sequence
+    ([150, 700, 33], [400, 650, 33], 4, 2, 64, torch.float16, False, (60, 30)),
 ]
 
 
