@@ -106,3 +106,18 @@ def test_varlen_rejects_bad_offsets_arguments(lib):
     assert args(0x60002, 0x60000, 2, 10, 10, 20, 20) == fa.FA_ERR_ALIGNMENT  # misaligned
     assert args(0x60000, 0x60000, 2, 30, 10, 20, 20) == fa.FA_ERR_INVALID_ARG  # max > total
     assert args(0x60000, 0x60000, 0, 10, 10, 20, 20) == fa.FA_ERR_INVALID_ARG  # no sequences
+
+
+@pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, 0.999, float("nan")])
+def test_dropout_rejects_bad_probability(lib, p):
+    # p outside [0, 1), or so close to 1 that round(256 (1 - p)) is 0: rejected
+    # before any CUDA call, by the dense and the packed-batch entry points alike
+    st3 = _strides(128 * 2 * 64, 2 * 64, 64)
+    rc = lib.fa_fwd_dropout(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 1, 128, 128, 2, 2, 64,
+                            st3, st3, st3, st3, 0, 0.125, 0, -1, -1, p, 7, 0, None)
+    assert rc == fa.FA_ERR_INVALID_ARG
+    st2 = (ctypes.c_int64 * 2)(256, 64)
+    rc = lib.fa_fwd_varlen_dropout(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x60000,
+                                   2, 10, 10, 20, 20, 4, 4, 64, st2, st2, st2, st2, 0, 0.125, 1,
+                                   -1, -1, p, 7, 0, None)
+    assert rc == fa.FA_ERR_INVALID_ARG
