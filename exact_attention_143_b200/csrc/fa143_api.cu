@@ -448,16 +448,16 @@ int check_varlen(const int* cu_q, const int* cu_k, int B, int max_q, int max_k, 
   return FA_OK;
 }
 
-}  // namespace
 
-extern "C" {
-
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
-           int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3], const int64_t k_stride[3],
-           const int64_t v_stride[3], const int64_t o_stride[3], int dtype, float softmax_scale,
-           int causal, int window_left, int window_right, void* stream) {
+// The dense and packed-batch forward entry points, with or without dropout
+// (dp = nullptr: none; head_dim 256 only without).
+int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+              int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3],
+              const int64_t k_stride[3], const int64_t v_stride[3], const int64_t o_stride[3],
+              int dtype, float softmax_scale, int causal, int window_left, int window_right,
+              void* stream, const fa::DropoutParams* dp) {
   int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right,
-                        true);
+                        dp == nullptr);
   if (rc) return rc;
   if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
   const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
@@ -466,18 +466,17 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
   return fwd_impl(tq, tk, tv, to, lse, size_t(B) * Hq * Nq * sizeof(float), B, Nq, Nk, Hq, Hkv,
                   d, nullptr, nullptr, 0, 0, dtype, softmax_scale, causal, window_left,
-                  window_right, stream);
+                  window_right, stream, dp);
 }
 
-int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
-                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
-                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d,
-                  const int64_t q_stride[2], const int64_t k_stride[2],
-                  const int64_t v_stride[2], const int64_t o_stride[2], int dtype,
-                  float softmax_scale, int causal, int window_left, int window_right,
-                  void* stream) {
+int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+               const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+               int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d,
+               const int64_t q_stride[2], const int64_t k_stride[2], const int64_t v_stride[2],
+               const int64_t o_stride[2], int dtype, float softmax_scale, int causal,
+               int window_left, int window_right, void* stream, const fa::DropoutParams* dp) {
   int rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale,
-                        window_left, window_right, true);
+                        window_left, window_right, dp == nullptr);
   if (rc) return rc;
   if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
                          total_k)))
@@ -490,7 +489,31 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
   return fwd_impl(tq, tk, tv, to, lse, size_t(Hq) * total_q * sizeof(float), B, max_seqlen_q,
                   max_seqlen_k, Hq, Hkv, d, cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype,
-                  softmax_scale, causal, window_left, window_right, stream);
+                  softmax_scale, causal, window_left, window_right, stream, dp);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+           int Nk, int Hq, int Hkv, int d, const int64_t q_stride[3], const int64_t k_stride[3],
+           const int64_t v_stride[3], const int64_t o_stride[3], int dtype, float softmax_scale,
+           int causal, int window_left, int window_right, void* stream) {
+  return fwd_dense(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride,
+                   dtype, softmax_scale, causal, window_left, window_right, stream, nullptr);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d,
+                  const int64_t q_stride[2], const int64_t k_stride[2],
+                  const int64_t v_stride[2], const int64_t o_stride[2], int dtype,
+                  float softmax_scale, int causal, int window_left, int window_right,
+                  void* stream) {
+  return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                    total_q, total_k, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride, dtype,
+                    softmax_scale, causal, window_left, window_right, stream, nullptr);
 }
 
 size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d) {
@@ -661,19 +684,19 @@ int bwd_impl(const TensorDesc& tq, const TensorDesc& tk, const TensorDesc& tv,
   return FA_OK;
 }
 
-}  // namespace
 
-extern "C" {
-
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-           const float* lse, void* dq, void* dk, void* dv, void* workspace,
-           size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
-           const int64_t q_stride[3], const int64_t k_stride[3], const int64_t v_stride[3],
-           const int64_t o_stride[3], const int64_t do_stride[3], const int64_t dq_stride[3],
-           const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
-           float softmax_scale, int causal, int window_left, int window_right, void* stream) {
+// The dense and packed-batch backward entry points, with or without dropout
+// (dp = nullptr: none; head_dim 256 only without).
+int bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* dout,
+              const float* lse, void* dq, void* dk, void* dv, void* workspace,
+              size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+              const int64_t q_stride[3], const int64_t k_stride[3], const int64_t v_stride[3],
+              const int64_t o_stride[3], const int64_t do_stride[3],
+              const int64_t dq_stride[3], const int64_t dk_stride[3],
+              const int64_t dv_stride[3], int dtype, float softmax_scale, int causal,
+              int window_left, int window_right, void* stream, const fa::DropoutParams* dp) {
   int rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right,
-                        true);
+                        dp == nullptr);
   if (rc) return rc;
   if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
       !dk_stride || !dv_stride)
@@ -688,21 +711,20 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   const TensorDesc tdv{dv, dv_stride[0], dv_stride[1], dv_stride[2], B, Nk, Hkv, d};
   return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(B) * Hq * Nq * sizeof(float),
                   workspace, workspace_bytes, B, Nq, Nk, Hq, Hkv, d, nullptr, nullptr, 0, 0,
-                  dtype, softmax_scale, causal, window_left, window_right, stream);
+                  dtype, softmax_scale, causal, window_left, window_right, stream, dp);
 }
 
-int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
-                  size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k,
-                  int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq,
-                  int Hkv, int d, const int64_t q_stride[2], const int64_t k_stride[2],
-                  const int64_t v_stride[2], const int64_t o_stride[2],
-                  const int64_t do_stride[2], const int64_t dq_stride[2],
-                  const int64_t dk_stride[2], const int64_t dv_stride[2], int dtype,
-                  float softmax_scale, int causal, int window_left, int window_right,
-                  void* stream) {
+int bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, void* workspace,
+               size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+               int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv,
+               int d, const int64_t q_stride[2], const int64_t k_stride[2],
+               const int64_t v_stride[2], const int64_t o_stride[2], const int64_t do_stride[2],
+               const int64_t dq_stride[2], const int64_t dk_stride[2],
+               const int64_t dv_stride[2], int dtype, float softmax_scale, int causal,
+               int window_left, int window_right, void* stream, const fa::DropoutParams* dp) {
   int rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale,
-                        window_left, window_right, true);
+                        window_left, window_right, dp == nullptr);
   if (rc) return rc;
   if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
                          total_k)))
@@ -722,7 +744,41 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
   return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(Hq) * total_q * sizeof(float),
                   workspace, workspace_bytes, B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d,
                   cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype, softmax_scale, causal,
-                  window_left, window_right, stream);
+                  window_left, window_right, stream, dp);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, void* workspace,
+           size_t workspace_bytes, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+           const int64_t q_stride[3], const int64_t k_stride[3], const int64_t v_stride[3],
+           const int64_t o_stride[3], const int64_t do_stride[3], const int64_t dq_stride[3],
+           const int64_t dk_stride[3], const int64_t dv_stride[3], int dtype,
+           float softmax_scale, int causal, int window_left, int window_right, void* stream) {
+  return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Nq, Nk, Hq,
+                   Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride, dk_stride,
+                   dv_stride, dtype, softmax_scale, causal, window_left, window_right, stream,
+                   nullptr);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                  int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq,
+                  int Hkv, int d, const int64_t q_stride[2], const int64_t k_stride[2],
+                  const int64_t v_stride[2], const int64_t o_stride[2],
+                  const int64_t do_stride[2], const int64_t dq_stride[2],
+                  const int64_t dk_stride[2], const int64_t dv_stride[2], int dtype,
+                  float softmax_scale, int causal, int window_left, int window_right,
+                  void* stream) {
+  return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens_q,
+                    cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d,
+                    q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride, dk_stride,
+                    dv_stride, dtype, softmax_scale, causal, window_left, window_right, stream,
+                    nullptr);
 }
 
 int fa_get_device_error(void* stream) {
@@ -1188,22 +1244,14 @@ int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* 
                    int window_left, int window_right, float dropout_p, uint64_t seed,
                    uint32_t offset, void* stream) {
   int T = 0;
-  int rc = dropout_threshold(dropout_p, &T);
+  const int rc = dropout_threshold(dropout_p, &T);
   if (rc) return rc;
   if (T >= 256)  // nothing is dropped
-    return fa_fwd(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride,
-                  dtype, softmax_scale, causal, window_left, window_right, stream);
-  rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
-  if (rc) return rc;
-  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
-  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
-  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
-  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
-  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
+    return fwd_dense(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride,
+                     dtype, softmax_scale, causal, window_left, window_right, stream, nullptr);
   const fa::DropoutParams dp = make_dropout(T, seed, offset);
-  return fwd_impl(tq, tk, tv, to, lse, size_t(B) * Hq * Nq * sizeof(float), B, Nq, Nk, Hq, Hkv,
-                  d, nullptr, nullptr, 0, 0, dtype, softmax_scale, causal, window_left,
-                  window_right, stream, &dp);
+  return fwd_dense(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride,
+                   dtype, softmax_scale, causal, window_left, window_right, stream, &dp);
 }
 
 int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -1216,30 +1264,17 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
                    float softmax_scale, int causal, int window_left, int window_right,
                    float dropout_p, uint64_t seed, uint32_t offset, void* stream) {
   int T = 0;
-  int rc = dropout_threshold(dropout_p, &T);
+  const int rc = dropout_threshold(dropout_p, &T);
   if (rc) return rc;
-  if (T >= 256)
-    return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Nq, Nk, Hq,
-                  Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride,
-                  dk_stride, dv_stride, dtype, softmax_scale, causal, window_left, window_right,
-                  stream);
-  rc = check_common(B, Nq, Nk, Hq, Hkv, d, dtype, softmax_scale, window_left, window_right);
-  if (rc) return rc;
-  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
-      !dk_stride || !dv_stride)
-    return FA_ERR_INVALID_ARG;
-  const TensorDesc tq{q, q_stride[0], q_stride[1], q_stride[2], B, Nq, Hq, d};
-  const TensorDesc tk{k, k_stride[0], k_stride[1], k_stride[2], B, Nk, Hkv, d};
-  const TensorDesc tv{v, v_stride[0], v_stride[1], v_stride[2], B, Nk, Hkv, d};
-  const TensorDesc to{o, o_stride[0], o_stride[1], o_stride[2], B, Nq, Hq, d};
-  const TensorDesc tdo{dout, do_stride[0], do_stride[1], do_stride[2], B, Nq, Hq, d};
-  const TensorDesc tdq{dq, dq_stride[0], dq_stride[1], dq_stride[2], B, Nq, Hq, d};
-  const TensorDesc tdk{dk, dk_stride[0], dk_stride[1], dk_stride[2], B, Nk, Hkv, d};
-  const TensorDesc tdv{dv, dv_stride[0], dv_stride[1], dv_stride[2], B, Nk, Hkv, d};
+  if (T >= 256)  // nothing is dropped
+    return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Nq, Nk, Hq,
+                     Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride,
+                     dk_stride, dv_stride, dtype, softmax_scale, causal, window_left, window_right,
+                     stream, nullptr);
   const fa::DropoutParams dp = make_dropout(T, seed, offset);
-  return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(B) * Hq * Nq * sizeof(float),
-                  workspace, workspace_bytes, B, Nq, Nk, Hq, Hkv, d, nullptr, nullptr, 0, 0,
-                  dtype, softmax_scale, causal, window_left, window_right, stream, &dp);
+  return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Nq, Nk, Hq,
+                   Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride, dk_stride,
+                   dv_stride, dtype, softmax_scale, causal, window_left, window_right, stream, &dp);
 }
 
 int fa_fwd_varlen_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -1250,29 +1285,16 @@ int fa_fwd_varlen_dropout(const void* q, const void* k, const void* v, void* o, 
                           float softmax_scale, int causal, int window_left, int window_right,
                           float dropout_p, uint64_t seed, uint32_t offset, void* stream) {
   int T = 0;
-  int rc = dropout_threshold(dropout_p, &T);
+  const int rc = dropout_threshold(dropout_p, &T);
   if (rc) return rc;
   if (T >= 256)  // nothing is dropped
-    return fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q,
-                         max_seqlen_k, total_q, total_k, Hq, Hkv, d, q_stride, k_stride,
-                         v_stride, o_stride, dtype, softmax_scale, causal, window_left,
-                         window_right, stream);
-  rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale, window_left,
-                    window_right);
-  if (rc) return rc;
-  if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
-                         total_k)))
-    return rc;
-  if (total_q > (1 << 28) || total_k > (1 << 28)) return FA_ERR_INVALID_ARG;
-  if (!q_stride || !k_stride || !v_stride || !o_stride || !lse) return FA_ERR_INVALID_ARG;
-  const TensorDesc tq{q, 0, q_stride[0], q_stride[1], 1, total_q, Hq, d};
-  const TensorDesc tk{k, 0, k_stride[0], k_stride[1], 1, total_k, Hkv, d};
-  const TensorDesc tv{v, 0, v_stride[0], v_stride[1], 1, total_k, Hkv, d};
-  const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
+    return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                      total_q, total_k, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride, dtype,
+                      softmax_scale, causal, window_left, window_right, stream, nullptr);
   const fa::DropoutParams dp = make_dropout(T, seed, offset);
-  return fwd_impl(tq, tk, tv, to, lse, size_t(Hq) * total_q * sizeof(float), B, max_seqlen_q,
-                  max_seqlen_k, Hq, Hkv, d, cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype,
-                  softmax_scale, causal, window_left, window_right, stream, &dp);
+  return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                    total_q, total_k, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride, dtype,
+                    softmax_scale, causal, window_left, window_right, stream, &dp);
 }
 
 int fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, const void* o,
@@ -1287,37 +1309,20 @@ int fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, const voi
                           float softmax_scale, int causal, int window_left, int window_right,
                           float dropout_p, uint64_t seed, uint32_t offset, void* stream) {
   int T = 0;
-  int rc = dropout_threshold(dropout_p, &T);
+  const int rc = dropout_threshold(dropout_p, &T);
   if (rc) return rc;
-  if (T >= 256)
-    return fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
-                         cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
-                         total_k, Hq, Hkv, d, q_stride, k_stride, v_stride, o_stride, do_stride,
-                         dq_stride, dk_stride, dv_stride, dtype, softmax_scale, causal,
-                         window_left, window_right, stream);
-  rc = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, dtype, softmax_scale, window_left,
-                    window_right);
-  if (rc) return rc;
-  if ((rc = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
-                         total_k)))
-    return rc;
-  if (total_q > (1 << 28) || total_k > (1 << 28)) return FA_ERR_INVALID_ARG;
-  if (!q_stride || !k_stride || !v_stride || !o_stride || !do_stride || !dq_stride ||
-      !dk_stride || !dv_stride)
-    return FA_ERR_INVALID_ARG;
-  const TensorDesc tq{q, 0, q_stride[0], q_stride[1], 1, total_q, Hq, d};
-  const TensorDesc tk{k, 0, k_stride[0], k_stride[1], 1, total_k, Hkv, d};
-  const TensorDesc tv{v, 0, v_stride[0], v_stride[1], 1, total_k, Hkv, d};
-  const TensorDesc to{o, 0, o_stride[0], o_stride[1], 1, total_q, Hq, d};
-  const TensorDesc tdo{dout, 0, do_stride[0], do_stride[1], 1, total_q, Hq, d};
-  const TensorDesc tdq{dq, 0, dq_stride[0], dq_stride[1], 1, total_q, Hq, d};
-  const TensorDesc tdk{dk, 0, dk_stride[0], dk_stride[1], 1, total_k, Hkv, d};
-  const TensorDesc tdv{dv, 0, dv_stride[0], dv_stride[1], 1, total_k, Hkv, d};
+  if (T >= 256)  // nothing is dropped
+    return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens_q,
+                      cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d,
+                      q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride, dk_stride,
+                      dv_stride, dtype, softmax_scale, causal, window_left, window_right, stream,
+                      nullptr);
   const fa::DropoutParams dp = make_dropout(T, seed, offset);
-  return bwd_impl(tq, tk, tv, to, tdo, tdq, tdk, tdv, lse, size_t(Hq) * total_q * sizeof(float),
-                  workspace, workspace_bytes, B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d,
-                  cu_seqlens_q, cu_seqlens_k, total_q, total_k, dtype, softmax_scale, causal,
-                  window_left, window_right, stream, &dp);
+  return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens_q,
+                    cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d,
+                    q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride, dk_stride,
+                    dv_stride, dtype, softmax_scale, causal, window_left, window_right, stream,
+                    &dp);
 }
 
 }  // extern "C"
