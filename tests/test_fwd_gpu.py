@@ -79,6 +79,14 @@ def test_gqa_window(d, dtype, Hq, Hkv, causal, window):
     run_case(2, 700, 700, Hq, Hkv, d, dtype, causal, window, seed=12)
 
 
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)], ids=["d64", "d128"])
+@pytest.mark.parametrize("Nq,Nk", [(333, 200), (200, 333), (1, 129)])
+def test_gqa_window_unequal_lengths(d, dtype, Nq, Nk):
+    # head-pair work tiles where some query tiles see no key at all (Nq > Nk
+    # with a causal window leaves the first Nq - Nk rows empty)
+    run_case(1, Nq, Nk, 4, 2, d, dtype, True, (100, 0), seed=13)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (8, 1), (6, 2)])
 def test_gqa(Hq, Hkv):
     run_case(2, 260, 260, Hq, Hkv, 128, torch.bfloat16, True, (-1, -1), seed=7)
