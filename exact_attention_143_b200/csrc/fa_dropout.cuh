@@ -53,7 +53,7 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
 // indexing, so no divergent branches.
 __device__ __forceinline__ void transpose4_lanes(uint32_t (&r)[4], int q) {
   const bool o1 = (q & 1) != 0, o2 = (q & 2) != 0;
-  // first exchange: entries k with bit 0 of k != bit 0 of q come from lane q ^ 1
+  // round 1: entries k with bit 0 of k != bit 0 of q come from lane q ^ 1
   uint32_t sa = o1 ? r[0] : r[1], sb = o1 ? r[2] : r[3];
   sa = __shfl_xor_sync(0xffffffffu, sa, 1);
   sb = __shfl_xor_sync(0xffffffffu, sb, 1);
@@ -64,7 +64,7 @@ __device__ __forceinline__ void transpose4_lanes(uint32_t (&r)[4], int q) {
     r[1] = sa;
     r[3] = sb;
   }
-  // second exchange: entries k with bit 1 of k != bit 1 of q come from lane q ^ 2
+  // round 2: entries k with bit 1 of k != bit 1 of q come from lane q ^ 2
   sa = o2 ? r[0] : r[2];
   sb = o2 ? r[1] : r[3];
   sa = __shfl_xor_sync(0xffffffffu, sa, 2);
