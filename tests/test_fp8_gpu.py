@@ -140,3 +140,29 @@ def test_fp8_workload_full_size_sampled():
         bound, var = fp8_error_model(q64, k64, v64, w.softmax_scale, w.causal, (-1, -1), b, h)
         parts.append(((b, slice(None), h, slice(None)), bound, var))
     check_fp8(o, o_ref, parts)
+
+
+def test_fp8_long_causal_full_size_sampled_blocks():
+    # the 16384-token causal d = 128 shape the bench times (where 2 of every 8
+    # exponential pairs take the FMA-pipe exp2); two 128-row query blocks of two
+    # heads are checked: a block's rows see keys [0, last row], so the oracle and
+    # the error model run on that block against its key prefix (bottom-right
+    # causal alignment keeps the same visibility)
+    w = FP8_WORKLOADS["fwd_fp8_1x16384_h16_d128_e4m3_causal"]
+    q8, k8, v8, q64, k64, v64 = fp8_inputs(w.batch, w.seqlen, w.seqlen, w.q_heads, w.kv_heads,
+                                           w.head_dim, w.descales, w.seed)
+    o, lse = fa.fa_fwd_fp8(q8.to(DEV), k8.to(DEV), v8.to(DEV), softmax_scale=w.softmax_scale,
+                           causal=w.causal, descale_q=w.descales[0], descale_k=w.descales[1],
+                           descale_v=w.descales[2])
+    torch.cuda.synchronize()
+    assert fa.get_device_error() == fa.FA_OK
+    o_cpu, lse_cpu = o.cpu(), lse.cpu()
+    for h in (3, 14):
+        for r0 in (8064, 16256):
+            r1 = r0 + 128
+            qs = q64[:, r0:r1, h:h + 1]
+            ks, vs = k64[:, :r1, h:h + 1], v64[:, :r1, h:h + 1]
+            ob, lb = oracle.attention_fwd(qs, ks, vs, w.softmax_scale, True)
+            check_lse(lse_cpu[:, h:h + 1, r0:r1], lb, "LSE[h %d, rows %d:%d]" % (h, r0, r1))
+            bound, var = fp8_error_model(qs, ks, vs, w.softmax_scale, True, (-1, -1), 0, 0)
+            check_fp8(o_cpu[:, r0:r1, h:h + 1], ob, [((0, slice(None), 0, slice(None)), bound, var)])
